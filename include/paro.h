@@ -1,0 +1,155 @@
+/*
+ * paro.h - C ABI of the B200 (sm_100a) rotated W4G128 linear layer.
+ *
+ * The layer (ParoQuant; CSDN article "ParoQuant", section 2.1, and the ICLR
+ * 2026 paper-notes page, "key design", final transform equation):
+ *
+ *     Y = (X T^-1) * dequant(Q(T W))^T,   T = R_K ... R_1 diag(alpha)
+ *
+ * R_t is a layer of independent Givens rotations over disjoint channel pairs
+ * that never leave their 128-channel quantisation group (paper notes,
+ * "independent rotation"); each pair (i, j) with angle th maps
+ * (v_i, v_j) -> (cos th v_i - sin th v_j, sin th v_i + cos th v_j)
+ * (CSDN article, section 2.2, the 2x2 matrix). Layer index 0 is applied
+ * first, on the weight side and on the activation side alike:
+ *     X T^-1 = X diag(1/alpha) R_1^T ... R_K^T.
+ * Q is asymmetric INT4 round-to-nearest per 128-input group (W4G128) with an
+ * fp16 scale s and an int4 zero z; dequant(q) = fp16((q - z) * s).
+ *
+ * Conventions for every entry point
+ *   - Tensors are row-major and contiguous. "in" is the input-feature count
+ *     (a multiple of 128), "out" the output-feature count (a multiple of 16),
+ *     "tokens" the number of activation rows.
+ *   - fp16 tensors are passed as void* / uint16_t* holding IEEE binary16.
+ *   - Pointers named *_dev are device pointers on the current CUDA device;
+ *     pointers named *_host are host pointers. The caller owns every buffer.
+ *   - Calls that take a stream enqueue work on it and return without
+ *     synchronising; the stream is a cudaStream_t (0 = legacy default stream).
+ *     Hot-path calls (paro_rotate, paro_linear) allocate nothing.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Every call returns a paro_status; on anything but PARO_OK,
+ *     paro_last_error() returns a message for the calling thread. Argument
+ *     errors are detected on the host before anything is enqueued.
+ */
+#ifndef PARO_H
+#define PARO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PARO_OK = 0,
+    PARO_ERR_ARG = 1,          /* invalid argument (null, size, alignment, pair table) */
+    PARO_ERR_UNSUPPORTED = 2,  /* valid but not supported by this build (e.g. group != 128) */
+    PARO_ERR_CUDA = 3,         /* a CUDA runtime call or a kernel launch failed */
+    PARO_ERR_DEVICE = 4        /* no usable sm_100 device */
+} paro_status;
+
+typedef void* paro_stream;     /* a cudaStream_t */
+
+/* Opaque prepared rotation: the device-resident form of (pairs, theta, alpha)
+ * for one linear layer. */
+typedef struct paro_rot paro_rot;
+
+/* Validate and prepare the scaled pairwise rotation T of one layer and upload
+ * it to the current device (setup; allocates device memory; synchronous).
+ *   in_features      multiple of `group`
+ *   group            channels per quantisation group; only 128 is supported
+ *   K                number of rotation layers, 0..16 (K = 0: T = diag(alpha))
+ *   pairs_per_group  P, 1..group/2 active pairs per (layer, group)
+ *   pairs_host       int16 [K][in/group][P][2], group-local channel indices
+ *                    (0..group-1); (i, j) order as in the 2x2 matrix above.
+ *                    Within one (layer, group) no channel may appear twice.
+ *   theta_host       float [K][in/group][P], radians
+ *   alpha_host       float [in_features], finite and non-zero
+ * Paper: ICLR 2026 notes, "key design" (Givens decomposition, independent
+ * rotation, K = 8 default, final transform T). */
+paro_status paro_rot_create(paro_rot** out, int64_t in_features, int group, int K,
+                            int pairs_per_group, const int16_t* pairs_host,
+                            const float* theta_host, const float* alpha_host);
+
+/* Free a handle from paro_rot_create (synchronous). NULL is accepted. */
+paro_status paro_rot_destroy(paro_rot* rot);
+
+/* Xr = X T^-1 (CSDN article, section 2.1: the activation side of
+ * Y = (X T^-1)(T W)): divide channel c by alpha_c, then apply layers
+ * t = 1..K with the 2x2 formula. fp32 arithmetic, fp16 in and out.
+ *   X_dev, Xr_dev  fp16 [tokens][in_features]; may not alias.
+ *   tokens >= 0 (0 is a no-op). */
+paro_status paro_rotate(const paro_rot* rot, const void* X_dev, void* Xr_dev,
+                        int64_t tokens, paro_stream stream);
+
+/* Sizes in bytes of the device weight format written by paro_pack_weights. */
+paro_status paro_pack_size(int64_t in_features, int64_t out_features,
+                           size_t* qweight_bytes, size_t* scales_bytes, size_t* zeros_bytes);
+
+/* Pack logical W4G128 tensors into the device weight format read by
+ * paro_linear (the int4 layout of the weight stream; one 16x16 tile is one
+ * 32-bit word per lane of a warp, nibbles ordered for a two-instruction
+ * int4->fp16 conversion).
+ *   q_dev      uint8  [out][in], values 0..15
+ *   s_dev      fp16   [out][in/128], the stored scales
+ *   z_dev      uint8  [out][in/128], values 0..15
+ *   qweight_dev, scales_dev, zeros_dev: outputs sized by paro_pack_size.
+ * Paper: W4G128 (paper notes, main-experiment table heading); s and z are the
+ * quantisation parameters named in the notes' training-strategy section. */
+paro_status paro_pack_weights(const uint8_t* q_dev, const uint16_t* s_dev, const uint8_t* z_dev,
+                              int64_t in_features, int64_t out_features,
+                              void* qweight_dev, void* scales_dev, void* zeros_dev,
+                              paro_stream stream);
+
+/* Expand the device weight format back to w_hat = fp16((q - z) * s),
+ * fp16 [out][in] (the dequantisation used inside paro_linear; exact product,
+ * one rounding). */
+paro_status paro_dequant(const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
+                         int64_t in_features, int64_t out_features, void* W_dev,
+                         paro_stream stream);
+
+/* Offline converter: W' = T W along the input axis (fp64), then asymmetric
+ * RTN per 128-input group: s = fp16((max-min)/15) floored at 2^-14,
+ * z = clamp(rint(-min/s), 0, 15), q = clamp(rint(w/s) + z, 0, 15).
+ *   W_dev  fp16 [out][in] (PyTorch orientation); outputs q_dev uint8 [out][in],
+ *   s_dev fp16 [out][in/128], z_dev uint8 [out][in/128].
+ * Paper: T W in the final-transform equation (paper notes, "key design");
+ * the RTN rule is this library's reading of W4G128. */
+paro_status paro_quantize_weights(const paro_rot* rot, const void* W_dev, int64_t out_features,
+                                  uint8_t* q_dev, uint16_t* s_dev, uint8_t* z_dev,
+                                  paro_stream stream);
+
+/* Bytes of workspace paro_linear needs for this shape. */
+paro_status paro_linear_workspace_size(int64_t tokens, int64_t in_features, int64_t out_features,
+                                       size_t* bytes);
+
+/* Y = (X T^-1) w_hat^T, fp32 accumulation, fp16 out (CSDN article,
+ * section 2.1, without the bias).
+ *   rot           prepared rotation, or NULL for the unrotated W4G128 layer
+ *                 (theta = 0, alpha = 1)
+ *   X_dev         fp16 [tokens][in_features]
+ *   qweight_dev, scales_dev, zeros_dev   from paro_pack_weights
+ *   Y_dev         fp16 [tokens][out_features]
+ *   workspace_dev at least paro_linear_workspace_size bytes, zero-filled
+ *                 before its first use. Its first
+ *                 paro_linear_workspace_size(16, in, out) bytes hold split-k
+ *                 accumulators that every call leaves zero-filled again; the
+ *                 rest (tokens > 16) is scratch for X T^-1. Calls that share a
+ *                 workspace must not overlap on the GPU.
+ * tokens <= 16 run the fused decode kernel (rotation in the prologue, int4
+ * weight stream); larger batches rotate into the workspace and run the
+ * tensor-core prefill GEMM. */
+paro_status paro_linear(const paro_rot* rot, const void* X_dev,
+                        const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
+                        void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,
+                        void* workspace_dev, size_t workspace_bytes, paro_stream stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* paro_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARO_H */

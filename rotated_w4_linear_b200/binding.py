@@ -1,0 +1,191 @@
+"""Thin ctypes binding of libparo.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: tensors are checked for dtype/device/contiguity and
+their data pointers are handed to the library together with torch's current
+CUDA stream. If the library is missing the import fails loudly; there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libparo.so")
+
+PARO_OK = 0
+_STATUS = {0: "PARO_OK", 1: "PARO_ERR_ARG", 2: "PARO_ERR_UNSUPPORTED", 3: "PARO_ERR_CUDA", 4: "PARO_ERR_DEVICE"}
+
+_lib: Optional[ctypes.CDLL] = None
+
+_vp, _i64, _int, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "paro_rot_create": [ctypes.POINTER(_vp), _i64, _int, _int, _int, _vp, _vp, _vp],
+    "paro_rot_destroy": [_vp],
+    "paro_rotate": [_vp, _vp, _vp, _i64, _vp],
+    "paro_pack_size": [_i64, _i64, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
+    "paro_pack_weights": [_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp],
+    "paro_dequant": [_vp, _vp, _vp, _i64, _i64, _vp, _vp],
+    "paro_quantize_weights": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
+    "paro_linear_workspace_size": [_i64, _i64, _i64, ctypes.POINTER(_sz)],
+    "paro_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
+    "paro_last_error": [],
+}
+
+
+class ParoError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libparo.so (built in-tree by rotated_w4_linear_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m rotated_w4_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_char_p if name == "paro_last_error" else ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, st: int) -> None:
+    if st != PARO_OK:
+        raise ParoError(fn, st, lib().paro_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class Rotation:
+    """Owner of a paro_rot handle (device-resident prepared rotation)."""
+
+    def __init__(self, pairs: np.ndarray, theta: np.ndarray, alpha: np.ndarray, group: int = 128):
+        pairs = np.ascontiguousarray(pairs, dtype=np.int16)
+        theta = np.ascontiguousarray(theta, dtype=np.float32)
+        alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+        K = int(pairs.shape[0]) if pairs.ndim == 4 else 0
+        P = int(pairs.shape[2]) if K else 0
+        self.in_features = int(alpha.shape[0])
+        self.K, self.P = K, P
+        h = _vp()
+        _check("paro_rot_create", lib().paro_rot_create(
+            ctypes.byref(h), self.in_features, group, K, P,
+            pairs.ctypes.data if K else None, theta.ctypes.data if K else None, alpha.ctypes.data))
+        self.handle = h
+
+    def close(self) -> None:
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            _check("paro_rot_destroy", lib().paro_rot_destroy(self.handle))
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def paro_rot_create(pairs, theta, alpha, group: int = 128) -> Rotation:
+    return Rotation(pairs, theta, alpha, group)
+
+
+def paro_rotate(rot: Rotation, X: torch.Tensor, Xr: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if Xr is None:
+        Xr = torch.empty_like(X)
+    _dev(X, torch.float16, "X"), _dev(Xr, torch.float16, "Xr")
+    if X.shape != Xr.shape or X.dim() != 2 or X.shape[1] != rot.in_features:
+        raise ValueError("X/Xr must be [tokens][in_features]")
+    _check("paro_rotate", lib().paro_rotate(rot.handle, X.data_ptr(), Xr.data_ptr(), X.shape[0], _stream(stream)))
+    return Xr
+
+
+def paro_pack_size(in_features: int, out_features: int):
+    q, s, z = _sz(), _sz(), _sz()
+    _check("paro_pack_size", lib().paro_pack_size(in_features, out_features, ctypes.byref(q), ctypes.byref(s), ctypes.byref(z)))
+    return q.value, s.value, z.value
+
+
+def paro_pack_weights(q: torch.Tensor, s: torch.Tensor, z: torch.Tensor, stream=None):
+    """Logical (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]) on the
+    device -> device format (qweight, scales, zeros) as uint8 tensors."""
+    out_f, in_f = q.shape
+    qb, sb, zb = paro_pack_size(in_f, out_f)
+    dev = q.device
+    qw = torch.empty(qb, dtype=torch.uint8, device=dev)
+    sp = torch.empty(sb, dtype=torch.uint8, device=dev)
+    zp = torch.empty(zb, dtype=torch.uint8, device=dev)
+    _check("paro_pack_weights", lib().paro_pack_weights(
+        _dev(q, torch.uint8, "q"), _dev(s, torch.float16, "s"), _dev(z, torch.uint8, "z"), in_f, out_f,
+        qw.data_ptr(), sp.data_ptr(), zp.data_ptr(), _stream(stream)))
+    return qw, sp, zp
+
+
+def paro_dequant(qw, sp, zp, in_features: int, out_features: int, stream=None) -> torch.Tensor:
+    W = torch.empty((out_features, in_features), dtype=torch.float16, device=qw.device)
+    _check("paro_dequant", lib().paro_dequant(_dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"),
+                                              _dev(zp, torch.uint8, "zeros"), in_features, out_features,
+                                              W.data_ptr(), _stream(stream)))
+    return W
+
+
+def paro_quantize_weights(rot: Rotation, W: torch.Tensor, stream=None):
+    """W fp16 [out][in] -> (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]) of T W."""
+    out_f, in_f = W.shape
+    G = in_f // 128
+    q = torch.empty((out_f, in_f), dtype=torch.uint8, device=W.device)
+    s = torch.empty((out_f, G), dtype=torch.float16, device=W.device)
+    z = torch.empty((out_f, G), dtype=torch.uint8, device=W.device)
+    _check("paro_quantize_weights", lib().paro_quantize_weights(
+        rot.handle, _dev(W, torch.float16, "W"), out_f, q.data_ptr(), s.data_ptr(), z.data_ptr(), _stream(stream)))
+    return q, s, z
+
+
+def paro_linear_workspace_size(tokens: int, in_features: int, out_features: int) -> int:
+    b = _sz()
+    _check("paro_linear_workspace_size", lib().paro_linear_workspace_size(tokens, in_features, out_features, ctypes.byref(b)))
+    return b.value
+
+
+def workspace(tokens: int, in_features: int, out_features: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace of the size paro_linear needs (allocated by torch)."""
+    n = paro_linear_workspace_size(tokens, in_features, out_features)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def paro_linear(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_features: int,
+                Y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    T, in_f = X.shape
+    if Y is None:
+        Y = torch.empty((T, out_features), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(T, in_f, out_features, X.device)
+    _check("paro_linear", lib().paro_linear(
+        rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
+        _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"),
+        _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
+        _stream(stream)))
+    return Y

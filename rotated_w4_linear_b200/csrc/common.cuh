@@ -1,0 +1,117 @@
+// Shared device helpers for the sm_100a kernels of the rotated W4G128 layer.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#define PARO_GROUP 128
+
+namespace paro {
+
+// ---------------------------------------------------------------------------
+// Prepared rotation parameters ("rotation block"), one per (layer t, group g),
+// 1152 bytes: 128 partner bytes, then 128 float2 (a, b).
+// Channel c of the group becomes a * v[c] + b * v[partner[c]]:
+//   first channel i of a pair (i, j, th): a = cos th, b = -sin th, partner j
+//   second channel j:                     a = cos th, b = +sin th, partner i
+//   channel in no pair:                   a = 1,      b = 0,       partner c
+// which is the 2x2 Givens matrix of the ParoQuant CSDN article (section 2.2)
+// written per output channel.
+// ---------------------------------------------------------------------------
+constexpr int kRotBlockBytes = 128 + 128 * 8;
+
+__device__ __forceinline__ const uint8_t* rot_block(const uint8_t* rotp, int t, int g, int G) {
+    return rotp + ((size_t)t * G + g) * kRotBlockBytes;
+}
+
+// ---------------------------------------------------------------------------
+// int4 weight format (Kernel 4). For row block rb (16 output rows) and 64-wide
+// k block kb, 512 bytes: lane L (g = L >> 2, q = L & 3) owns 16 bytes = 4 words,
+// word j covering the 16x16 tile k in [64 kb + 16 j, +16). The word's nibbles:
+//   n0 (g,   4q)   n4 (g,   4q+1)   n1 (g,   4q+2)   n5 (g,   4q+3)
+//   n2 (g+8, 4q)   n6 (g+8, 4q+1)   n3 (g+8, 4q+2)   n7 (g+8, 4q+3)
+// (row within the block, k within the tile). Nibbles i and i+4 sit 16 bits
+// apart, so one LOP3 turns them into the fp16 pair (1024 + n_i, 1024 + n_i+4).
+// Scales: uint32 [out/16][G][8], word g = (s[row g] | s[row g+8] << 16).
+// Zeros:  uint8  [out/16][G][8], byte g = (z[row g] | z[row g+8] << 4).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t nib_pair_to_f16x2(uint32_t w) {
+    // (w & 0x000f000f) | 0x64006400: fp16 bit patterns of 1024 + nibble
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x000f000fu), "r"(0x64006400u));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2_rn(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_rn(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// zero byte (z0 | z1 << 4) -> fp16x2 (1024 + z, 1024 + z) for z0 (lo) and z1 (hi)
+__device__ __forceinline__ void zero_bias(uint32_t zbyte, uint32_t& zb0, uint32_t& zb1) {
+    zb0 = ((zbyte & 0xFu) | 0x6400u) * 0x00010001u;
+    zb1 = (((zbyte >> 4) & 0xFu) | 0x6400u) * 0x00010001u;
+}
+
+// scale word (s0 | s1 << 16) -> (s0, s0) and (s1, s1)
+__device__ __forceinline__ void scale_pairs(uint32_t sw, uint32_t& sc0, uint32_t& sc1) {
+    sc0 = __byte_perm(sw, sw, 0x1010);
+    sc1 = __byte_perm(sw, sw, 0x3232);
+}
+
+// One packed word -> four fp16x2 of w_hat = fp16((q - z) * s):
+//   h[0] = (g,   k0, k0+1)   h[1] = (g,   k0+2, k0+3)
+//   h[2] = (g+8, k0, k0+1)   h[3] = (g+8, k0+2, k0+3)
+// (1024+q) - (1024+z) is exact in fp16; the product is rounded once.
+__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb0, uint32_t sc0,
+                                             uint32_t zb1, uint32_t sc1, uint32_t h[4]) {
+    h[0] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w), zb0), sc0);
+    h[1] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w >> 4), zb0), sc0);
+    h[2] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w >> 8), zb1), sc1);
+    h[3] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w >> 12), zb1), sc1);
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---------------------------------------------------------------------------
+// One warp rotates one 128-channel group of one token held as 4 channels per
+// lane (lane L: channels 4L..4L+3). `buf` is 128 floats of warp-private shared
+// memory. Applies layers t = 0..K-1 of group g.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void rotate_group_warp(float v[4], const uint8_t* rotp, int g, int G, int K,
+                                                  float* buf, int lane) {
+    for (int t = 0; t < K; ++t) {
+        const uint8_t* blk = rot_block(rotp, t, g, G);
+        const uint32_t pw = __ldg(reinterpret_cast<const uint32_t*>(blk) + lane);
+        const float4 c01 = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane);
+        const float4 c23 = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane + 1);
+        *reinterpret_cast<float4*>(buf + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
+        __syncwarp();
+        const float p0 = buf[pw & 0xFF], p1 = buf[(pw >> 8) & 0xFF];
+        const float p2 = buf[(pw >> 16) & 0xFF], p3 = buf[pw >> 24];
+        __syncwarp();
+        v[0] = fmaf(c01.y, p0, c01.x * v[0]);
+        v[1] = fmaf(c01.w, p1, c01.z * v[1]);
+        v[2] = fmaf(c23.y, p2, c23.x * v[2]);
+        v[3] = fmaf(c23.w, p3, c23.z * v[3]);
+    }
+}
+
+}  // namespace paro

@@ -1,0 +1,35 @@
+// Host-side launchers of the sm_100a kernels (internal to libparo).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace paro {
+
+struct RotDev {
+    int64_t in = 0;         // input features
+    int G = 0;              // groups of 128
+    int K = 0;              // rotation layers
+    int P = 0;              // active pairs per (layer, group)
+    uint8_t* rotp = nullptr;       // [K][G] rotation blocks (fp32 coefficients)
+    float* inv_alpha = nullptr;    // [in] fp32 1/alpha
+    uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
+    double* alpha64 = nullptr;     // [in] alpha as fp64
+};
+
+cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
+
+cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out,
+                        void* qw, void* scp, void* zp, cudaStream_t s);
+cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int64_t in, int64_t out,
+                           void* W, cudaStream_t s);
+cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t* q, uint16_t* sc,
+                            uint8_t* z, cudaStream_t s);
+
+// Fused decode GEMV (tokens <= 16). rot may be null (no rotation).
+size_t gemv_workspace_bytes(int64_t T, int64_t in, int64_t out);
+cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
+                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes,
+                        cudaStream_t s);
+
+}  // namespace paro

@@ -1,0 +1,282 @@
+// Host side of the C ABI declared in include/paro.h: argument validation,
+// preparation of the rotation parameters, dispatch by token count.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/paro.h"
+#include "common.cuh"
+#include "kernels.h"
+
+struct paro_rot {
+    paro::RotDev dev;
+    int device = 0;
+    void* block = nullptr;   // single device allocation holding every table
+};
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+paro_status fail(paro_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+paro_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(PARO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The kernels are built for sm_100a only; refuse anything else up front.
+paro_status check_device() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+        return fail(PARO_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev, major, minor);
+    return PARO_OK;
+}
+
+paro_status check_shape(int64_t in, int64_t out) {
+    if (in <= 0 || in % 128) return fail(PARO_ERR_ARG, "in_features=%lld must be a positive multiple of 128", (long long)in);
+    if (out <= 0 || out % 16) return fail(PARO_ERR_ARG, "out_features=%lld must be a positive multiple of 16", (long long)out);
+    if (in > (1LL << 20) || out > (1LL << 22)) return fail(PARO_ERR_UNSUPPORTED, "shape too large");
+    return PARO_OK;
+}
+
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+}  // namespace
+
+extern "C" {
+
+const char* paro_last_error(void) { return g_err; }
+
+paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P, const int16_t* pairs,
+                            const float* theta, const float* alpha) {
+    g_err[0] = 0;
+    if (!out) return fail(PARO_ERR_ARG, "out is null");
+    *out = nullptr;
+    if (group != 128) return fail(PARO_ERR_UNSUPPORTED, "group=%d: only 128 is supported", group);
+    if (in <= 0 || in % group) return fail(PARO_ERR_ARG, "in_features=%lld must be a positive multiple of %d", (long long)in, group);
+    if (in > (1LL << 20)) return fail(PARO_ERR_UNSUPPORTED, "in_features too large");
+    if (K < 0 || K > 16) return fail(PARO_ERR_ARG, "K=%d must be in 0..16", K);
+    if (K > 0 && (P < 1 || P > group / 2)) return fail(PARO_ERR_ARG, "pairs_per_group=%d must be in 1..%d", P, group / 2);
+    if (!alpha) return fail(PARO_ERR_ARG, "alpha is null");
+    if (K > 0 && (!pairs || !theta)) return fail(PARO_ERR_ARG, "pairs/theta is null");
+    paro_status st = check_device();
+    if (st != PARO_OK) return st;
+
+    const int G = (int)(in / group);
+    for (int64_t c = 0; c < in; ++c)
+        if (!std::isfinite(alpha[c]) || alpha[c] == 0.0f)
+            return fail(PARO_ERR_ARG, "alpha[%lld] must be finite and non-zero", (long long)c);
+
+    // host images of the tables
+    std::vector<uint8_t> rot32((size_t)K * G * paro::kRotBlockBytes);
+    std::vector<uint8_t> rot64((size_t)K * G * (128 + 128 * 16));
+    for (int t = 0; t < K; ++t) {
+        for (int g = 0; g < G; ++g) {
+            uint8_t partner[128];
+            float a32[128], b32[128];
+            double a64[128], b64[128];
+            bool used[128] = {false};
+            for (int c = 0; c < 128; ++c) { partner[c] = (uint8_t)c; a32[c] = 1.f; b32[c] = 0.f; a64[c] = 1.0; b64[c] = 0.0; }
+            for (int p = 0; p < P; ++p) {
+                const size_t base = (((size_t)t * G + g) * P + p);
+                const int i = pairs[2 * base], j = pairs[2 * base + 1];
+                const float th = theta[base];
+                if (i < 0 || i >= group || j < 0 || j >= group)
+                    return fail(PARO_ERR_ARG, "pair (%d,%d) of layer %d group %d leaves the group", i, j, t, g);
+                if (i == j || used[i] || used[j])
+                    return fail(PARO_ERR_ARG, "channel reused within layer %d group %d (pair %d: %d,%d)", t, g, p, i, j);
+                if (!std::isfinite(th)) return fail(PARO_ERR_ARG, "theta of layer %d group %d pair %d is not finite", t, g, p);
+                used[i] = used[j] = true;
+                const double c = std::cos((double)th), s = std::sin((double)th);
+                partner[i] = (uint8_t)j; a64[i] = c; b64[i] = -s;
+                partner[j] = (uint8_t)i; a64[j] = c; b64[j] = s;
+                a32[i] = (float)c; b32[i] = (float)(-s);
+                a32[j] = (float)c; b32[j] = (float)s;
+            }
+            uint8_t* b = &rot32[((size_t)t * G + g) * paro::kRotBlockBytes];
+            memcpy(b, partner, 128);
+            for (int c = 0; c < 128; ++c) {
+                memcpy(b + 128 + 8 * c, &a32[c], 4);
+                memcpy(b + 128 + 8 * c + 4, &b32[c], 4);
+            }
+            uint8_t* b6 = &rot64[((size_t)t * G + g) * (128 + 128 * 16)];
+            memcpy(b6, partner, 128);
+            for (int c = 0; c < 128; ++c) {
+                memcpy(b6 + 128 + 16 * c, &a64[c], 8);
+                memcpy(b6 + 128 + 16 * c + 8, &b64[c], 8);
+            }
+        }
+    }
+    std::vector<float> inv_alpha((size_t)in);
+    std::vector<double> alpha64((size_t)in);
+    for (int64_t c = 0; c < in; ++c) {
+        inv_alpha[c] = (float)(1.0 / (double)alpha[c]);
+        alpha64[c] = (double)alpha[c];
+    }
+
+    const size_t o_rot32 = 0;
+    const size_t o_inv = o_rot32 + round256(rot32.size());
+    const size_t o_rot64 = o_inv + round256(inv_alpha.size() * sizeof(float));
+    const size_t o_a64 = o_rot64 + round256(rot64.size());
+    const size_t total = o_a64 + round256(alpha64.size() * sizeof(double));
+
+    paro_rot* r = new (std::nothrow) paro_rot();
+    if (!r) return fail(PARO_ERR_ARG, "out of host memory");
+    cudaGetDevice(&r->device);
+    cudaError_t e = cudaMalloc(&r->block, total);
+    if (e != cudaSuccess) { delete r; return cuda_fail(e, "cudaMalloc(rotation tables)"); }
+    char* base = static_cast<char*>(r->block);
+    e = cudaMemcpy(base + o_rot32, rot32.data(), rot32.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + o_inv, inv_alpha.data(), inv_alpha.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + o_rot64, rot64.data(), rot64.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(r->block); delete r; return cuda_fail(e, "cudaMemcpy(rotation tables)"); }
+    r->dev.in = in;
+    r->dev.G = G;
+    r->dev.K = K;
+    r->dev.P = P;
+    r->dev.rotp = reinterpret_cast<uint8_t*>(base + o_rot32);
+    r->dev.inv_alpha = reinterpret_cast<float*>(base + o_inv);
+    r->dev.rotp64 = reinterpret_cast<uint8_t*>(base + o_rot64);
+    r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);
+    *out = r;
+    return PARO_OK;
+}
+
+paro_status paro_rot_destroy(paro_rot* r) {
+    g_err[0] = 0;
+    if (!r) return PARO_OK;
+    cudaError_t e = cudaFree(r->block);
+    delete r;
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "cudaFree(rotation tables)");
+}
+
+paro_status paro_rotate(const paro_rot* r, const void* X, void* Xr, int64_t T, paro_stream stream) {
+    g_err[0] = 0;
+    if (!r) return fail(PARO_ERR_ARG, "rot is null");
+    if (T < 0) return fail(PARO_ERR_ARG, "tokens=%lld < 0", (long long)T);
+    if (T == 0) return PARO_OK;
+    if (!X || !Xr) return fail(PARO_ERR_ARG, "X/Xr is null");
+    if (!aligned16(X) || !aligned16(Xr)) return fail(PARO_ERR_ARG, "X/Xr must be 16-byte aligned");
+    if (X == Xr) return fail(PARO_ERR_ARG, "X and Xr must not alias");
+    if (T > (1LL << 31) / r->dev.in) return fail(PARO_ERR_UNSUPPORTED, "tokens too large");
+    cudaError_t e = paro::launch_rotate(r->dev, X, Xr, T, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "rotate launch");
+}
+
+paro_status paro_pack_size(int64_t in, int64_t out, size_t* qb, size_t* sb, size_t* zb) {
+    g_err[0] = 0;
+    paro_status st = check_shape(in, out);
+    if (st != PARO_OK) return st;
+    if (!qb || !sb || !zb) return fail(PARO_ERR_ARG, "null size pointer");
+    *qb = (size_t)(in * out / 2);
+    *sb = (size_t)((out / 16) * (in / 128) * 8 * 4);
+    *zb = (size_t)((out / 16) * (in / 128) * 8);
+    return PARO_OK;
+}
+
+paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t* z, int64_t in, int64_t out,
+                              void* qw, void* sp, void* zp, paro_stream stream) {
+    g_err[0] = 0;
+    paro_status st = check_shape(in, out);
+    if (st != PARO_OK) return st;
+    if (!q || !s || !z || !qw || !sp || !zp) return fail(PARO_ERR_ARG, "null pointer");
+    if (!aligned16(qw) || !aligned16(sp) || !aligned16(zp)) return fail(PARO_ERR_ARG, "outputs must be 16-byte aligned");
+    cudaError_t e = paro::launch_pack(q, s, z, in, out, qw, sp, zp, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "pack launch");
+}
+
+paro_status paro_dequant(const void* qw, const void* sp, const void* zp, int64_t in, int64_t out, void* W,
+                         paro_stream stream) {
+    g_err[0] = 0;
+    paro_status st = check_shape(in, out);
+    if (st != PARO_OK) return st;
+    if (!qw || !sp || !zp || !W) return fail(PARO_ERR_ARG, "null pointer");
+    if (!aligned16(qw) || !aligned16(sp) || !aligned16(W)) return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
+    cudaError_t e = paro::launch_dequant(qw, sp, zp, in, out, W, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "dequant launch");
+}
+
+paro_status paro_quantize_weights(const paro_rot* r, const void* W, int64_t out, uint8_t* q, uint16_t* s,
+                                  uint8_t* z, paro_stream stream) {
+    g_err[0] = 0;
+    if (!r) return fail(PARO_ERR_ARG, "rot is null");
+    paro_status st = check_shape(r->dev.in, out);
+    if (st != PARO_OK) return st;
+    if (!W || !q || !s || !z) return fail(PARO_ERR_ARG, "null pointer");
+    if (!aligned16(W) || !aligned16(q)) return fail(PARO_ERR_ARG, "W/q must be 16-byte aligned");
+    cudaError_t e = paro::launch_quantize(r->dev, W, out, q, s, z, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "quantize launch");
+}
+
+paro_status paro_linear_workspace_size(int64_t T, int64_t in, int64_t out, size_t* bytes) {
+    g_err[0] = 0;
+    paro_status st = check_shape(in, out);
+    if (st != PARO_OK) return st;
+    if (T < 0 || !bytes) return fail(PARO_ERR_ARG, "bad tokens or null bytes");
+    size_t b = round256(paro::gemv_workspace_bytes(16, in, out));
+    if (T > 16) b += round256((size_t)T * in * 2);     // X' for the prefill path
+    *bytes = b;
+    return PARO_OK;
+}
+
+paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp, void* Y,
+                        int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes, paro_stream stream) {
+    g_err[0] = 0;
+    paro_status st = check_shape(in, out);
+    if (st != PARO_OK) return st;
+    if (T < 0) return fail(PARO_ERR_ARG, "tokens=%lld < 0", (long long)T);
+    if (T == 0) return PARO_OK;
+    if (r && r->dev.in != in) return fail(PARO_ERR_ARG, "rotation prepared for in=%lld, layer has in=%lld", (long long)r->dev.in, (long long)in);
+    if (!X || !qw || !sp || !zp || !Y || !ws) return fail(PARO_ERR_ARG, "null pointer");
+    if (!aligned16(X) || !aligned16(qw) || !aligned16(sp) || !aligned16(zp) || !aligned16(Y) || !aligned16(ws))
+        return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
+    if (T > (1LL << 31) / in) return fail(PARO_ERR_UNSUPPORTED, "tokens too large");
+    size_t need = 0;
+    paro_linear_workspace_size(T, in, out, &need);
+    if (ws_bytes < need) return fail(PARO_ERR_ARG, "workspace_bytes=%zu < %zu", ws_bytes, need);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const paro::RotDev* rd = r ? &r->dev : nullptr;
+    cudaError_t e;
+    if (T <= 16) {
+        e = paro::launch_gemv(rd, X, qw, sp, zp, Y, T, in, out, ws, ws_bytes, s);
+        return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
+    }
+    // prefill: X' into the workspace, then the contraction over 16-token slices
+    char* gws = static_cast<char*>(ws);
+    const size_t gbytes = round256(paro::gemv_workspace_bytes(16, in, out));
+    void* xr = gws + gbytes;
+    const void* src = X;
+    if (r) {
+        e = paro::launch_rotate(r->dev, X, xr, T, s);
+        if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
+        src = xr;
+    }
+    for (int64_t t0 = 0; t0 < T; t0 += 16) {
+        const int64_t n = (T - t0 < 16) ? (T - t0) : 16;
+        e = paro::launch_gemv(nullptr, static_cast<const char*>(src) + t0 * in * 2, qw, sp, zp,
+                              static_cast<char*>(Y) + t0 * out * 2, n, in, out, gws, gbytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    }
+    return PARO_OK;
+}
+
+}  // extern "C"

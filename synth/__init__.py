@@ -98,6 +98,22 @@ def rotation_params(in_features: int, K: int, seed: int, pairs_per_group: int = 
             channel_scales(in_features, seed))
 
 
+_S_CODES = 7
+
+
+def w4_codes(out_features: int, in_features: int, seed: int, group: int = GROUP):
+    """Random valid W4G128 codes, not derived from any weight: q uint8 [out][in]
+    ~ U{0..15}, z uint8 [out][in/group] ~ U{0..15}, s fp16 [out][in/group]
+    ~ U(0.002, 0.02). Used where a test needs the layer's inputs at full size
+    without running the offline quantiser."""
+    rng = _rng(seed, _S_CODES)
+    G = in_features // group
+    q = rng.integers(0, 16, (out_features, in_features), dtype=np.uint8)
+    z = rng.integers(0, 16, (out_features, G), dtype=np.uint8)
+    s = rng.uniform(0.002, 0.02, (out_features, G)).astype(np.float16)
+    return q, s, z
+
+
 def layer_seed(config_id: int, layer_id: int) -> int:
     """Seed convention: 1000 * config id + layer id."""
     return 1000 * int(config_id) + int(layer_id)

@@ -1,0 +1,68 @@
+"""The C-ABI library loads and exports every entry point include/paro.h
+declares; host-only calls validate their arguments (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "paro.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(paro_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from rotated_w4_linear_b200 import build, binding
+    build.build()
+    return binding.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert "paro_rotate" in names and "paro_linear" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_binding_names_match_header():
+    from rotated_w4_linear_b200 import binding
+    for n in _declared():
+        assert n in binding._SIGS, n
+
+
+def test_pack_size(L):
+    from rotated_w4_linear_b200 import binding
+    qb, sb, zb = binding.paro_pack_size(4096, 6144)
+    assert qb == 4096 * 6144 // 2
+    assert sb == 6144 // 16 * 32 * 8 * 4 and zb == 6144 // 16 * 32 * 8
+    # 0.5 + 2/128 + 0.5/128 bytes per weight
+    assert (qb + sb + zb) / (4096 * 6144) == pytest.approx(0.5 + 2 / 128 + 0.5 / 128)
+
+
+@pytest.mark.parametrize("inf,outf", [(100, 64), (128, 20), (0, 16), (-128, 16)])
+def test_bad_shapes_rejected(L, inf, outf):
+    from rotated_w4_linear_b200 import binding
+    with pytest.raises(binding.ParoError) as e:
+        binding.paro_pack_size(inf, outf)
+    assert e.value.status == 1
+    assert "must be" in L.paro_last_error().decode()
+
+
+def test_null_arguments_rejected_before_any_launch(L):
+    assert L.paro_rotate(None, None, None, 4, None) == 1
+    assert b"rot is null" in L.paro_last_error()
+    assert L.paro_linear(None, None, None, None, None, None, 4, 256, 64, None, 0, None) == 1
+    b = ctypes.c_size_t()
+    assert L.paro_linear_workspace_size(16, 4096, 4096, ctypes.byref(b)) == 0 and b.value > 0
+    assert L.paro_rot_create(None, 256, 128, 8, 64, None, None, None) == 1
+    assert L.paro_rot_destroy(None) == 0
+
+
+def test_unsupported_group(L):
+    h = ctypes.c_void_p()
+    assert L.paro_rot_create(ctypes.byref(h), 256, 64, 8, 32, None, None, None) == 2

@@ -1,0 +1,221 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU fp64 oracle.
+
+Tolerances (stated by the task for this layer, with the readings of the
+open points):
+  * int4 unpack/dequant: bit-exact fp16;
+  * offline quantiser: bit-exact q, s, z;
+  * rotated activations: per-element relative error <= 1e-3 against fp64,
+    the denominator floored at 1% of the element's group maximum;
+  * layer output: ||Y - Y_ref|| / ||Y_ref|| <= 2e-3 and max |Y - Y_ref| <=
+    max(1e-2, floor + 2e-3), where `floor` is the max error of the ideal fp16
+    pipeline (X' rounded to fp16, exact contraction, Y rounded to fp16): a
+    kernel with fp16 activations and outputs cannot beat it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import paro_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B(cuda_lib):
+    from rotated_w4_linear_b200 import binding
+    return binding
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+ROT_TOL = 1e-3
+REL_TOL = 2e-3
+ABS_TOL = 1e-2
+
+
+def check_rotation(got16, x, pairs, theta, alpha):
+    ref = O.rotate_activations(x, pairs, theta, alpha)
+    fl, lit = O.rotation_rel_error(got16.astype(np.float64), ref)
+    assert fl <= ROT_TOL, (fl, lit)
+    return fl
+
+
+def check_linear(y16, x, pairs, theta, alpha, q, s, z):
+    if pairs is None:                       # unrotated layer: theta = 0, alpha = 1
+        pairs, theta, alpha = synth.rotation_params(x.shape[1], 1, 0)
+        theta = np.zeros_like(theta)
+        alpha = np.ones_like(alpha)
+    ref = O.linear(x, pairs, theta, alpha, q, s, z)
+    ideal = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z)
+    rel, mx = O.output_errors(y16.astype(np.float64), ref)
+    _, floor = O.output_errors(ideal.astype(np.float64), ref)
+    assert rel <= REL_TOL, (rel, mx, floor)
+    assert mx <= max(ABS_TOL, floor + 2e-3), (rel, mx, floor)
+    return rel, mx, floor
+
+
+# ---------------------------------------------------------------- rotation
+@pytest.mark.parametrize("T,in_f,K,P", [
+    (16, 512, 8, 64),      # the tiny single layer
+    (1, 4096, 8, 64),
+    (3, 4096, 1, 64),
+    (17, 4096, 4, 64),
+    (256, 4096, 8, 13),    # partial matchings: 13 of 64 pairs per group
+    (9, 384, 8, 64),       # ragged token tile, odd group count
+    (5, 256, 0, 1),        # K = 0: channel scaling only
+])
+def test_rotate_parity(B, T, in_f, K, P):
+    seed = synth.layer_seed(1, T + K)
+    pairs, theta, alpha = synth.rotation_params(in_f, max(K, 1), seed, pairs_per_group=P)
+    if K == 0:
+        pairs, theta = pairs[:0], theta[:0]
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    got = host(B.paro_rotate(rot, dev(x)))
+    check_rotation(got, x, pairs, theta, alpha)
+
+
+@pytest.mark.parametrize("T", [2048, 8192])
+def test_rotate_full_size_sampled_rows(B, T):
+    seed = synth.layer_seed(1, T)
+    pairs, theta, alpha = synth.rotation_params(4096, 8, seed)
+    x = synth.activations(T, 4096, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    got = host(B.paro_rotate(rot, dev(x)))
+    rows = np.random.default_rng(T).choice(T, 64, replace=False)
+    rows[0], rows[-1] = 0, T - 1
+    check_rotation(got[rows], x[rows], pairs, theta, alpha)
+
+
+def test_rotate_empty_and_invalid(B):
+    pairs, theta, alpha = synth.rotation_params(256, 2, 1)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    x = torch.empty((0, 256), dtype=torch.float16, device="cuda")
+    assert B.paro_rotate(rot, x).shape == (0, 256)
+    bad = pairs.copy()
+    bad[1, 0, 3, 1] = bad[1, 0, 2, 0]
+    with pytest.raises(B.ParoError):
+        B.paro_rot_create(bad, theta, alpha)
+    with pytest.raises(B.ParoError):
+        B.paro_rot_create(pairs, theta, np.zeros_like(alpha))
+
+
+# ---------------------------------------------------------------- int4 format
+@pytest.mark.parametrize("out_f,in_f", [(48, 384), (6144, 4096), (4096, 14336)])
+def test_pack_dequant_bit_exact(B, out_f, in_f):
+    q, s, z = synth.w4_codes(out_f, in_f, seed=out_f + in_f)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    got = host(B.paro_dequant(qw, sp, zp, in_f, out_f))
+    ref = O.dequantize(q, s, z)
+    assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+
+
+def test_dequant_all_codes_and_extreme_scales(B):
+    # every (q, z) pair, scales spanning the fp16 normal range
+    out_f, in_f = 16, 256 * 2
+    q = np.tile(np.arange(16, dtype=np.uint8), (out_f, in_f // 16))
+    z = (np.arange(out_f * 4).reshape(out_f, 4) % 16).astype(np.uint8)
+    s = np.array([[2.0 ** -14, 0.000123, 0.75, 4095.0]] * out_f, np.float16)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    got = host(B.paro_dequant(qw, sp, zp, in_f, out_f))
+    assert np.array_equal(got.view(np.uint16), O.dequantize(q, s, z).view(np.uint16))
+
+
+# ---------------------------------------------------------------- converter
+@pytest.mark.parametrize("out_f,in_f,K,P", [(64, 512, 8, 64), (256, 4096, 8, 64), (32, 384, 4, 13)])
+def test_quantize_matches_oracle(B, out_f, in_f, K, P):
+    seed = synth.layer_seed(0, out_f + K)
+    pairs, theta, alpha = synth.rotation_params(in_f, K, seed, pairs_per_group=P)
+    w = synth.weight(out_f, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    q, s, z = (host(t) for t in B.paro_quantize_weights(rot, dev(w)))
+    q0, s0, z0, _ = O.quantize_layer(w, pairs, theta, alpha)
+    assert np.array_equal(s.view(np.uint16), s0.view(np.uint16))
+    assert np.array_equal(z, z0)
+    assert np.array_equal(q, q0)
+
+
+# ---------------------------------------------------------------- the layer
+def _layer(B, in_f, out_f, K, P, seed, oracle_quant=True):
+    pairs, theta, alpha = synth.rotation_params(in_f, K, seed, pairs_per_group=P)
+    if oracle_quant:
+        w = synth.weight(out_f, in_f, seed)
+        q, s, z, _ = O.quantize_layer(w, pairs, theta, alpha)
+    else:
+        q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    return (pairs, theta, alpha, q, s, z), (qw, sp, zp)
+
+
+@pytest.mark.parametrize("T,in_f,out_f,K,P", [
+    (16, 512, 512, 8, 64),     # the tiny single layer, every output
+    (1, 512, 512, 8, 64),
+    (3, 384, 48, 8, 64),
+    (8, 256, 80, 4, 13),
+    (9, 384, 48, 1, 64),
+    (17, 512, 96, 8, 64),      # > 16 tokens: prefill path
+    (40, 384, 48, 8, 64),
+])
+def test_linear_parity_exhaustive(B, T, in_f, out_f, K, P):
+    seed = synth.layer_seed(0, T * 7 + K)
+    (pairs, theta, alpha, q, s, z), (qw, sp, zp) = _layer(B, in_f, out_f, K, P, seed)
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    ws = B.workspace(T, in_f, out_f)
+    for _ in range(2):                 # twice: the accumulators must come back zeroed
+        y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f, ws=ws))
+        check_linear(y, x, pairs, theta, alpha, q, s, z)
+    acc_region = B.paro_linear_workspace_size(16, in_f, out_f)   # split-k accumulators + counters
+    assert int(ws[:acc_region].count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_linear_unrotated(B, T):
+    in_f, out_f = 512, 128
+    q, s, z = synth.w4_codes(out_f, in_f, seed=T)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed=T)
+    y = host(B.paro_linear(None, dev(x), qw, sp, zp, out_f))
+    check_linear(y, x, None, None, None, q, s, z)
+
+
+LLAMA = [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096)]
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+@pytest.mark.parametrize("in_f,out_f", LLAMA)
+def test_linear_decode_full_size_sampled(B, T, in_f, out_f):
+    seed = synth.layer_seed(2, in_f + out_f + T)
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+    q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
+    rows = np.random.default_rng(seed).choice(out_f, 256, replace=False)
+    rows[0], rows[-1] = 0, out_f - 1
+    check_linear(y[:, rows], x, pairs, theta, alpha, q[rows], s[rows], z[rows])
+
+
+@pytest.mark.parametrize("in_f,out_f", [(4096, 4096), (14336, 4096)])
+def test_linear_prefill_full_size_sampled(B, in_f, out_f):
+    T = 2048
+    seed = synth.layer_seed(3, in_f + out_f)
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+    q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
+    rng = np.random.default_rng(seed)
+    toks = rng.choice(T, 24, replace=False)
+    toks[0], toks[-1] = 0, T - 1
+    rows = rng.choice(out_f, 256, replace=False)
+    check_linear(y[np.ix_(toks, rows)], x[toks], pairs, theta, alpha, q[rows], s[rows], z[rows])

@@ -1,0 +1,391 @@
+"""Benchmark of the rotated W4G128 linear layer on B200.
+
+A step is one pass of the whole hot path (activation scaling, K Givens
+layers, int4 dequant and the contraction, all inside paro_linear) through
+every W4G128 projection of LAYERS distinct Llama-3-8B-shaped decoder layers
+(fused QKV 4096->6144, O 4096->4096, fused gate+up 4096->28672,
+down 14336->4096; K = 8 rotation layers, 64 pairs per group) for one decode
+batch of TOKENS synthetic tokens. LAYERS copies make each step's weights
+(4 x 113 MB) larger than the 126 MB L2, so no step reads weights from L2.
+
+value = algorithmic HBM bytes of all ranks / max-over-ranks device time:
+per projection 0.5195 B per weight (int4 q + fp16 s + int4 z per 128), the
+fp16 activations read and outputs written, and the rotation parameters
+(per pair one fp32 cos/sin pair and two channel bytes, plus 1/alpha).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--tokens T] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "ParoQuant W4G128 linear: decode HBM GB/s, prefill TFLOP/s, % of roofline"
+PROJ = [("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672), ("down", 14336, 4096)]
+K_LAYERS = 8
+GROUP = 128
+
+
+def weight_bytes(n_in, n_out):
+    return n_in * n_out // 2 + (n_out * n_in // GROUP) * 2 + (n_out * n_in // GROUP) // 2
+
+
+def rot_param_bytes(n_in, K=K_LAYERS, P=64):
+    return K * (n_in // GROUP) * P * (8 + 2) + 4 * n_in
+
+
+def call_bytes(T, n_in, n_out):
+    return weight_bytes(n_in, n_out) + 2 * T * n_in + 2 * T * n_out + rot_param_bytes(n_in)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for ln in f:
+                    p = [x.strip() for x in ln.split(",")]
+                    if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                        rows.append(p)
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# --------------------------------------------------------------------------- oracle baseline
+def cpu_baseline(tokens: int, budget_s: float = 12.0):
+    """The CPU fp64 oracle as it stands, on a bounded sample: whole projections
+    of layer 0 (every output row), one after another until ~budget_s."""
+    from oracle import paro_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    done_bytes, t_total, n_calls, names = 0, 0.0, 0, []
+    for i, (name, n_in, n_out) in enumerate(PROJ):
+        seed = synth.layer_seed(2, i)
+        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
+        q, s, z = synth.w4_codes(n_out, n_in, seed)
+        x = synth.activations(tokens, n_in, seed)
+        t0 = time.perf_counter()
+        O.linear(x, pairs, theta, alpha, q, s, z)
+        t_total += time.perf_counter() - t0
+        done_bytes += call_bytes(tokens, n_in, n_out)
+        n_calls += 1
+        names.append(name)
+        if t_total > budget_s:
+            break
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{n_calls} projections ({'+'.join(names)}) of one layer, every output row, "
+                      f"{tokens} tokens, fp64 numpy ({t_total:.1f} s)"}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    step_bytes = sum(call_bytes(args.tokens, i, o) for _, i, o in PROJ)
+    from oracle import paro_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    # one step of the reference arm: the four projections of one layer with
+    # 1/16 of their output rows (a bounded sample of the GPU arm's step)
+    inputs = []
+    for i, (name, n_in, n_out) in enumerate(PROJ):
+        seed = synth.layer_seed(2, i)
+        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
+        q, s_, z = synth.w4_codes(n_out // 16, n_in, seed)
+        x = synth.activations(args.tokens, n_in, seed)
+        inputs.append((x, pairs, theta, alpha, q, s_, z))
+    times = []
+    for k in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        for inp in inputs:
+            O.linear(*inp)
+        if k >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sample_bytes = sum(call_bytes(args.tokens, i, o // 16) for _, i, o in PROJ)
+    v = sample_bytes * len(times) / sum(times) / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config(args),
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
+                             "sample": "each step: the four projections of one layer with 1/16 of the output "
+                                       f"rows, {args.tokens} tokens (step bytes {sample_bytes} of {step_bytes})"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config(args):
+    return {"workload": f"llama3-8b decoder-layer W4G128 linears (qkv 4096x6144, o 4096x4096, "
+                        f"gate_up 4096x28672, down 14336x4096), decode {args.tokens} tokens, "
+                        f"K={K_LAYERS} rotation layers x 64 pairs/group",
+            "tokens": args.tokens, "layers_per_step": args.layers, "rotation_layers": K_LAYERS,
+            "group": GROUP, "l2": f"inputs larger than L2: {args.layers} distinct layers per step",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+# --------------------------------------------------------------------------- rotation alone
+def bench_rotate(args, torch, B, local):
+    """paro_rotate on X [tokens][4096] (fp16 in, fp16 out), distinct inputs per
+    call so that each step moves more than L2. Bytes: X read + X' written +
+    rotation parameters."""
+    torch.cuda.set_device(local)
+    T, n_in, K, P = args.tokens, 4096, args.rot_k, args.rot_pairs
+    pairs, theta, alpha = synth.rotation_params(n_in, K, synth.layer_seed(1, K), pairs_per_group=P)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    copies = max(1, (512 << 20) // (4 * T * n_in))
+    xs = [torch.from_numpy(synth.activations(T, n_in, synth.layer_seed(1, c))).cuda() for c in range(copies)]
+    ys = [torch.empty_like(x) for x in xs]
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        for x, y in zip(xs, ys):
+            B.paro_rotate(rot, x, y)
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(args.steps):
+        for x, y in zip(xs, ys):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            B.paro_rotate(rot, x, y)
+            e1.record(stream)
+            evs.append((e0, e1))
+    torch.cuda.synchronize()
+    per = sum(a.elapsed_time(b) for a, b in evs) / 1e3 / len(evs)
+    nbytes = 4 * T * n_in + K * (n_in // GROUP) * P * 10 + 4 * n_in
+    hbm_peak, _, kind = peaks()
+    print(json.dumps({"workload": f"paro_rotate tokens={T} hidden={n_in} K={K} pairs/group={P}",
+                      "us_per_call": per * 1e6, "GB/s": nbytes / per / 1e9,
+                      "roofline": {"bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm_peak,
+                                   "frac": nbytes / per / 1e9 / hbm_peak, "peak_source": kind},
+                      "copies": copies}), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--tokens", type=int, default=16)
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--impl", default="paro", choices=["paro", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="decode", choices=["decode", "rotate"],
+                    help="decode: the headline step; rotate: paro_rotate alone (hidden 4096)")
+    ap.add_argument("--rot-k", type=int, default=8)
+    ap.add_argument("--rot-pairs", type=int, default=64)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    from rotated_w4_linear_b200 import binding as B
+
+    if args.workload == "rotate":
+        return bench_rotate(args, torch, B, local)
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    T = args.tokens
+    dev = torch.device("cuda", local)
+    # ---- setup (untimed): per layer copy and projection, rotation + RTN on the GPU
+    layers = []
+    for l in range(args.layers):
+        projs = []
+        for i, (name, n_in, n_out) in enumerate(PROJ):
+            seed = synth.layer_seed(2, 100 * (rank * args.layers + l) + i)
+            pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
+            rot = B.paro_rot_create(pairs, theta, alpha)
+            w = torch.from_numpy(synth.weight(n_out, n_in, seed)).to(dev)
+            q, s, z = B.paro_quantize_weights(rot, w)
+            qw, sp, zp = B.paro_pack_weights(q, s, z)
+            del w, q, s, z
+            x = torch.from_numpy(synth.activations(T, n_in, seed)).to(dev)
+            y = torch.empty((T, n_out), dtype=torch.float16, device=dev)
+            ws = B.workspace(T, n_in, n_out, dev)
+            projs.append(dict(name=name, n_in=n_in, n_out=n_out, rot=rot, qw=qw, sp=sp, zp=zp, x=x, y=y, ws=ws))
+        layers.append(projs)
+    torch.cuda.synchronize()
+    calls = [p for projs in layers for p in projs]
+    step_bytes = sum(call_bytes(T, p["n_in"], p["n_out"]) for p in calls)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        for j, p in enumerate(calls):
+            if events is not None:
+                events[j][0].record(stream)
+            B.paro_linear(p["rot"], p["x"], p["qw"], p["sp"], p["zp"], p["n_out"], Y=p["y"], ws=p["ws"])
+            if events is not None:
+                events[j][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: device time of K steps
+    hbm_peak, _, peak_kind = peaks()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_index = vis.split(",")[local].strip() if vis else str(local)
+    with ClockSampler(smi_index) as clk:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+              for _ in range(args.steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(ev[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    clocks = clk.summary()
+
+    # per-launch durations of the decode kernel (one launch per paro_linear call)
+    kern_s = sum(e0.elapsed_time(e1) for evs in ev for (e0, e1) in evs) / 1e3
+    n_launch = args.steps * len(calls)
+
+    # ---- e2e: same step through host buffers (pinned), copies inside the timed region
+    xh = [torch.empty_like(p["x"], device="cpu").pin_memory() for p in calls]
+    yh = [torch.empty_like(p["y"], device="cpu").pin_memory() for p in calls]
+    for h, p in zip(xh, calls):
+        h.copy_(p["x"].cpu())
+    h2d = sum(h.numel() * 2 for h in xh)
+    d2h = sum(h.numel() * 2 for h in yh)
+
+    def e2e_step():
+        for h, p in zip(xh, calls):
+            p["x"].copy_(h, non_blocking=True)
+        step()
+        for h, p in zip(yh, calls):
+            h.copy_(p["y"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_elapsed = e0.elapsed_time(e1) / 1e3
+
+    if dist:
+        t = torch.tensor([elapsed, e2e_elapsed, kern_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed, e2e_elapsed, kern_s = (float(v) for v in t.tolist())
+
+    total_bytes = step_bytes * args.steps * world
+    value = total_bytes / elapsed / 1e9
+    achieved = step_bytes * args.steps / kern_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 (int4 weights, fp32 accumulate)",
+        "data": "synthetic (seeded Llama-3-8B-shaped layers; weights quantised on the GPU from T W)",
+        "config": config(args),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "gemv_kernel (fused decode)",
+                     "peak_source": f"{peak_kind} hbm_gbs"},
+        "e2e": {"value": step_bytes * args.steps * world / e2e_elapsed / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": n_launch,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(T)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for projs in layers:
+        for p in projs:
+            p["rot"].close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

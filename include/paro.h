@@ -131,15 +131,14 @@ paro_status paro_linear_workspace_size(int64_t tokens, int64_t in_features, int6
  *   X_dev         fp16 [tokens][in_features]
  *   qweight_dev, scales_dev, zeros_dev   from paro_pack_weights
  *   Y_dev         fp16 [tokens][out_features]
- *   workspace_dev at least paro_linear_workspace_size bytes, zero-filled
- *                 before its first use. Its first
- *                 paro_linear_workspace_size(16, in, out) bytes hold split-k
- *                 accumulators that every call leaves zero-filled again; the
- *                 rest (tokens > 16) is scratch for X T^-1. Calls that share a
- *                 workspace must not overlap on the GPU.
- * tokens <= 16 run the fused decode kernel (rotation in the prologue, int4
- * weight stream); larger batches rotate into the workspace and run the
- * tensor-core prefill GEMM. */
+ *   workspace_dev at least paro_linear_workspace_size bytes of scratch (no
+ *                 initialisation needed); it receives X T^-1 in fp16. Calls
+ *                 that share a workspace must not overlap on the GPU.
+ * The rotation kernel writes X T^-1 into the workspace; the contraction runs
+ * as a programmatic dependent launch of it (its weight loads start before
+ * the rotation has finished). tokens <= 16 use the int4 decode kernel
+ * (split-k reduced through distributed shared memory inside a thread-block
+ * cluster); larger batches use the tensor-core prefill GEMM. */
 paro_status paro_linear(const paro_rot* rot, const void* X_dev,
                         const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
                         void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,

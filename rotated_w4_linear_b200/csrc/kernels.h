@@ -26,8 +26,8 @@ cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int6
 cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t* q, uint16_t* sc,
                             uint8_t* z, cudaStream_t s);
 
-// Fused decode GEMV (tokens <= 16). rot may be null (no rotation).
-size_t gemv_workspace_bytes(int64_t T, int64_t in, int64_t out);
+// Decode path (tokens <= 16): rotation into ws (when rot is not null), then
+// the int4 GEMV launched as a programmatic dependent of it.
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
                         void* Y, int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes,
                         cudaStream_t s);

@@ -232,9 +232,7 @@ paro_status paro_linear_workspace_size(int64_t T, int64_t in, int64_t out, size_
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
     if (T < 0 || !bytes) return fail(PARO_ERR_ARG, "bad tokens or null bytes");
-    size_t b = round256(paro::gemv_workspace_bytes(16, in, out));
-    if (T > 16) b += round256((size_t)T * in * 2);     // X' for the prefill path
-    *bytes = b;
+    *bytes = round256((size_t)(T < 16 ? 16 : T) * in * 2);   // X T^-1 (fp16)
     return PARO_OK;
 }
 
@@ -261,19 +259,16 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
     // prefill: X' into the workspace, then the contraction over 16-token slices
-    char* gws = static_cast<char*>(ws);
-    const size_t gbytes = round256(paro::gemv_workspace_bytes(16, in, out));
-    void* xr = gws + gbytes;
     const void* src = X;
     if (r) {
-        e = paro::launch_rotate(r->dev, X, xr, T, s);
+        e = paro::launch_rotate(r->dev, X, ws, T, s);
         if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
-        src = xr;
+        src = ws;
     }
     for (int64_t t0 = 0; t0 < T; t0 += 16) {
         const int64_t n = (T - t0 < 16) ? (T - t0) : 16;
         e = paro::launch_gemv(nullptr, static_cast<const char*>(src) + t0 * in * 2, qw, sp, zp,
-                              static_cast<char*>(Y) + t0 * out * 2, n, in, out, gws, gbytes, s);
+                              static_cast<char*>(Y) + t0 * out * 2, n, in, out, nullptr, 0, s);
         if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     }
     return PARO_OK;

@@ -18,6 +18,9 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
                                                      int64_t T, int in, int G, int K,
                                                      const uint8_t* __restrict__ rotp,
                                                      const float* __restrict__ inv_alpha) {
+    // a kernel launched after this one on the stream may start now; it waits
+    // for this grid's completion before it reads Xr
+    asm volatile("griddepcontrol.launch_dependents;");
     __shared__ __align__(16) float buf[4][TT][128];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t task = (int64_t)blockIdx.x * 4 + warp;
@@ -41,25 +44,38 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
     }
 
     float(*b)[128] = buf[warp];
-    for (int t = 0; t < K; ++t) {
-        const uint8_t* blk = rot_block(rotp, t, g, G);
-        const uint32_t pw = __ldg(reinterpret_cast<const uint32_t*>(blk) + lane);
-        const float4 c01 = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane);
-        const float4 c23 = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane + 1);
-        const int p0 = pw & 0xFF, p1 = (pw >> 8) & 0xFF, p2 = (pw >> 16) & 0xFF, p3 = pw >> 24;
+    for (int tb = 0; tb < K; tb += 8) {
+        // all parameter loads of up to 8 layers are issued before any is used
+        uint32_t pw[8];
+        float4 c01[8], c23[8];
 #pragma unroll
-        for (int i = 0; i < TT; ++i)
-            *reinterpret_cast<float4*>(&b[i][4 * lane]) = make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < TT; ++i) {
-            const float q0 = b[i][p0], q1 = b[i][p1], q2 = b[i][p2], q3 = b[i][p3];
-            v[i][0] = fmaf(c01.y, q0, c01.x * v[i][0]);
-            v[i][1] = fmaf(c01.w, q1, c01.z * v[i][1]);
-            v[i][2] = fmaf(c23.y, q2, c23.x * v[i][2]);
-            v[i][3] = fmaf(c23.w, q3, c23.z * v[i][3]);
+        for (int u = 0; u < 8; ++u) {
+            if (tb + u < K) {
+                const uint8_t* blk = rot_block(rotp, tb + u, g, G);
+                pw[u] = __ldg(reinterpret_cast<const uint32_t*>(blk) + lane);
+                c01[u] = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane);
+                c23[u] = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane + 1);
+            }
         }
-        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (tb + u < K) {
+                const int p0 = pw[u] & 0xFF, p1 = (pw[u] >> 8) & 0xFF, p2 = (pw[u] >> 16) & 0xFF, p3 = pw[u] >> 24;
+#pragma unroll
+                for (int i = 0; i < TT; ++i)
+                    *reinterpret_cast<float4*>(&b[i][4 * lane]) = make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < TT; ++i) {
+                    const float q0 = b[i][p0], q1 = b[i][p1], q2 = b[i][p2], q3 = b[i][p3];
+                    v[i][0] = fmaf(c01[u].y, q0, c01[u].x * v[i][0]);
+                    v[i][1] = fmaf(c01[u].w, q1, c01[u].z * v[i][1]);
+                    v[i][2] = fmaf(c23[u].y, q2, c23[u].x * v[i][2]);
+                    v[i][3] = fmaf(c23[u].w, q3, c23[u].z * v[i][3]);
+                }
+                __syncwarp();
+            }
+        }
     }
 
 #pragma unroll
@@ -75,11 +91,17 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
 
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    constexpr int TT = 8;
-    const int64_t tasks = ((T + TT - 1) / TT) * r.G;
-    const int64_t blocks = (tasks + 3) / 4;
-    rotate_kernel<TT><<<(unsigned)blocks, 128, 0, s>>>(static_cast<const __half*>(X), static_cast<__half*>(Xr), T,
-                                                       (int)r.in, r.G, r.K, r.rotp, r.inv_alpha);
+    const __half* x = static_cast<const __half*>(X);
+    __half* y = static_cast<__half*>(Xr);
+    if (T <= 16) {   // decode batches: 4 tokens per warp for more warps in flight
+        constexpr int TT = 4;
+        const int64_t tasks = ((T + TT - 1) / TT) * r.G;
+        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotp, r.inv_alpha);
+    } else {
+        constexpr int TT = 8;
+        const int64_t tasks = ((T + TT - 1) / TT) * r.G;
+        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotp, r.inv_alpha);
+    }
     return cudaGetLastError();
 }
 

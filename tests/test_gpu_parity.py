@@ -169,11 +169,10 @@ def test_linear_parity_exhaustive(B, T, in_f, out_f, K, P):
     x = synth.activations(T, in_f, seed)
     rot = B.paro_rot_create(pairs, theta, alpha)
     ws = B.workspace(T, in_f, out_f)
-    for _ in range(2):                 # twice: the accumulators must come back zeroed
+    ws.fill_(0xA5)                     # scratch: any initial content
+    for _ in range(2):
         y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f, ws=ws))
         check_linear(y, x, pairs, theta, alpha, q, s, z)
-    acc_region = B.paro_linear_workspace_size(16, in_f, out_f)   # split-k accumulators + counters
-    assert int(ws[:acc_region].count_nonzero()) == 0
 
 
 @pytest.mark.parametrize("T", [1, 5, 16])

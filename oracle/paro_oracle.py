@@ -176,12 +176,14 @@ def linear(x: np.ndarray, pairs, theta, alpha, q, s, z, group: int = GROUP) -> n
     return xr @ dequantize(q, s, z, group).astype(np.float64).T
 
 
-def linear_fp16_pipeline(x: np.ndarray, pairs, theta, alpha, q, s, z, group: int = GROUP) -> np.ndarray:
+def linear_fp16_pipeline(x: np.ndarray, pairs, theta, alpha, q, s, z, group: int = GROUP,
+                         round_output: bool = True) -> np.ndarray:
     """The ideal fp16 pipeline: X' rounded to fp16, fp64 contraction with w_hat,
-    Y rounded to fp16. Its distance to `linear` is the format floor of any
-    kernel that stores X' and Y in fp16."""
+    Y rounded to fp16 (or left in fp64 with round_output=False). Its distance
+    to `linear` is the format floor of any kernel that stores X' and Y in fp16."""
     xr = rotate_activations(x, pairs, theta, alpha, group).astype(np.float16).astype(np.float64)
-    return (xr @ dequantize(q, s, z, group).astype(np.float64).T).astype(np.float16)
+    y = xr @ dequantize(q, s, z, group).astype(np.float64).T
+    return y.astype(np.float16) if round_output else y
 
 
 # --------------------------------------------------------------------------

@@ -33,7 +33,8 @@ __device__ __forceinline__ const uint8_t* rot_block(const uint8_t* rotp, int t, 
 // (row within the block, k within the tile). Nibbles i and i+4 sit 16 bits
 // apart, so one LOP3 turns them into the fp16 pair (1024 + n_i, 1024 + n_i+4).
 // Scales: uint32 [out/16][G][8], word g = (s[row g] | s[row g+8] << 16).
-// Zeros:  uint8  [out/16][G][8], byte g = (z[row g] | z[row g+8] << 4).
+// Zeros:  uint8  [out/16][Gp][8] with Gp = G rounded up to even (two groups'
+//         zeros form one aligned 16-byte copy), byte g = (z[row g] | z[row g+8] << 4).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t nib_pair_to_f16x2(uint32_t w) {
     // (w & 0x000f000f) | 0x64006400: fp16 bit patterns of 1024 + nibble
@@ -54,6 +55,34 @@ __device__ __forceinline__ uint32_t hmul2_rn(uint32_t a, uint32_t b) {
     return r;
 }
 
+__device__ __forceinline__ uint32_t hfma2_rn(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t w, uint32_t mask, uint32_t bits) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(mask), "r"(bits));
+    return r;
+}
+
+// Per-row zero constants from the zero byte (z0 | z1 << 4), as fp16x2 pairs:
+//   zb = (1024 + z, 1024 + z)   subtracted from (1024 + q)
+//   zc = -(64 + z, 64 + z)      added to (1024 + 16 q) / 16
+struct Zero2 {
+    uint32_t zb0, zc0, zb1, zc1;
+};
+__device__ __forceinline__ Zero2 zero_consts(uint32_t zbyte) {
+    const uint32_t z0 = zbyte & 0xFu, z1 = (zbyte >> 4) & 0xFu;
+    Zero2 r;
+    r.zb0 = (0x6400u | z0) * 0x00010001u;
+    r.zb1 = (0x6400u | z1) * 0x00010001u;
+    r.zc0 = (0xD400u | (z0 << 4)) * 0x00010001u;
+    r.zc1 = (0xD400u | (z1 << 4)) * 0x00010001u;
+    return r;
+}
+
 // zero byte (z0 | z1 << 4) -> fp16x2 (1024 + z, 1024 + z) for z0 (lo) and z1 (hi)
 __device__ __forceinline__ void zero_bias(uint32_t zbyte, uint32_t& zb0, uint32_t& zb1) {
     zb0 = ((zbyte & 0xFu) | 0x6400u) * 0x00010001u;
@@ -69,13 +98,40 @@ __device__ __forceinline__ void scale_pairs(uint32_t sw, uint32_t& sc0, uint32_t
 // One packed word -> four fp16x2 of w_hat = fp16((q - z) * s):
 //   h[0] = (g,   k0, k0+1)   h[1] = (g,   k0+2, k0+3)
 //   h[2] = (g+8, k0, k0+1)   h[3] = (g+8, k0+2, k0+3)
-// (1024+q) - (1024+z) is exact in fp16; the product is rounded once.
-__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb0, uint32_t sc0,
-                                             uint32_t zb1, uint32_t sc1, uint32_t h[4]) {
-    h[0] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w), zb0), sc0);
-    h[1] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w >> 4), zb0), sc0);
-    h[2] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w >> 8), zb1), sc1);
-    h[3] = hmul2_rn(hsub2_rn(nib_pair_to_f16x2(w >> 12), zb1), sc1);
+// Nibbles at bits 0-3 / 16-19 become 1024 + q under mask 0x000f000f, and
+// (1024 + q) - (1024 + z) = q - z exactly. Nibbles at bits 4-7 / 20-23 become
+// 1024 + 16 q under mask 0x00f000f0 (still inside the fp16 mantissa), and one
+// fma (1024 + 16 q) * 1/16 - (64 + z) = q - z is exact as well. One shift by
+// 8 serves the upper byte of each half. The product with s is rounded once.
+__device__ __forceinline__ void dequant_word(uint32_t w, const Zero2& z, uint32_t sc0, uint32_t sc1,
+                                             uint32_t h[4]) {
+    const uint32_t kMagic = 0x64006400u, kSixteenth = 0x2C002C00u;   // fp16x2 1024, 1/16
+    const uint32_t w8 = w >> 8;
+    h[0] = hmul2_rn(hsub2_rn(lop3_and_or(w, 0x000F000Fu, kMagic), z.zb0), sc0);
+    h[1] = hmul2_rn(hfma2_rn(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, z.zc0), sc0);
+    h[2] = hmul2_rn(hsub2_rn(lop3_and_or(w8, 0x000F000Fu, kMagic), z.zb1), sc1);
+    h[3] = hmul2_rn(hfma2_rn(lop3_and_or(w8, 0x00F000F0u, kMagic), kSixteenth, z.zc1), sc1);
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {

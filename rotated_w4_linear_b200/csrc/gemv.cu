@@ -5,23 +5,26 @@
 // Launch: a grid of (nsplit, rowtiles) CTAs of 8 warps; CTAs with the same
 // row tile form one thread-block cluster along x, each owning a k-chunk of
 // KC 128-channel groups. The kernel is launched with programmatic stream
-// serialisation, so it starts while the rotation kernel still runs:
-//   1. every warp issues the int4 loads of its first work item;
-//   2. griddepcontrol.wait: the rotation grid has completed and X' is
-//      visible; the CTA copies its X' chunk (all tokens) into shared memory;
-//   3. items (row block of 16 rows x 4 groups) are spread over the warps:
-//      each 32-bit int4 word becomes an m16n8k16 A fragment of the exact
-//      integers (q - z) in fp16 (LOP3 into the 1024 + q bit pattern, one exact
-//      fp16 subtraction); the B fragment (four consecutive channels of one
-//      token) comes from shared memory; each group's products are summed in
-//      fp32 by the tensor core (two independent accumulator chains) and then
-//      multiplied by the group's fp32 scale, i.e. the contraction uses the
-//      exact product (q - z) * s; the next item's loads are in flight
-//      meanwhile; per-item partial sums are added into a shared fp32 tile
-//      [token][row];
-//   4. split-k: the cluster's CTAs read each other's tiles through
-//      distributed shared memory; CTA x sums and stores the x-th slice of
-//      the rows as fp16. No global atomics and no workspace.
+// serialisation, so it starts while the rotation kernel still runs.
+//
+//   weight stream: warp w of a CTA owns the row blocks w, w + 8, ... of the
+//     tile, each over the whole k-chunk, as a sequence of items (16 rows x two
+//     groups: 2 KB of int4 codes + scales + zeros) streamed through a private
+//     3-stage shared-memory ring with cp.async (16-byte global->shared copies
+//     that bypass the registers): one commit group per item, wait on the
+//     oldest, so two items are in flight while one is consumed;
+//   X': after griddepcontrol.wait (the rotation grid has completed) the CTA
+//     copies its X' chunk (all tokens, zero rows >= T) into shared memory;
+//   math: each 32-bit int4 word is dequantised in registers (LOP3 into the
+//     1024 + q bit pattern, exact fp16 subtraction of 1024 + z, one rounded
+//     fp16 multiply: w_hat = fp16((q - z) s)) straight into an m16n8k16 A
+//     fragment; the B fragment (four consecutive channels of one token) comes
+//     from shared memory; fp32 accumulation in two independent chains;
+//   split-k: a row block's fp32 sums stay in registers over the chunk and
+//     are then stored into the CTA's shared tile [token][row]; after a
+//     cluster barrier CTA x sums its slice of the rows over the cluster's
+//     tiles with distributed shared memory loads and stores it as fp16. No
+//     global atomics, no workspace.
 // The k order inside each 16x16 tile follows the packed layout: the MMA's
 // logical k slot 2q+e holds channel 4q+e and slot 2q+8+e channel 4q+2+e.
 #include <algorithm>
@@ -34,15 +37,19 @@ namespace paro {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kItemGroups = 4;            // groups per work item
-constexpr int kItemBlocks = 2 * kItemGroups;  // 64-wide k blocks per item
+constexpr int kStages = 3;
+constexpr int kItemGroups = 2;                            // groups per item
+constexpr int kItemQBytes = kItemGroups * 2 * 512;        // int4 codes
+constexpr int kItemBytes = kItemQBytes + kItemGroups * 32 + 16;   // + scales + zeros
+constexpr int kMaxRbPerWarp = 4;                          // row blocks a warp keeps sums for
 
 struct GemvArgs {
     const __half* Xr;     // [T][in] fp16, already rotated
-    int T, in, out, G;
+    int T, in, out, G, Gp;
     int KC;               // groups per k-chunk (last chunk may be shorter)
     int RT;               // row blocks per CTA
     int nsplit;           // k-chunks = cluster size along x
+    int share;            // rows of the tile each cluster CTA finalises (multiple of 16)
     const uint4* qw;
     const uint32_t* sp;
     const uint8_t* zp;
@@ -57,42 +64,44 @@ __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t cta_rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(cta_rank));
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
     return v;
 }
-
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-struct Item {
-    uint4 w[kItemBlocks];
-    uint32_t s[kItemGroups];
-    uint32_t z[kItemGroups];
-};
-
-// Issue the loads of one item: row block rb, groups [g0, g0 + ng) (ng <= 4).
-__device__ __forceinline__ void load_item(Item& it, const GemvArgs& a, int rb, int g0, int ng, int lane) {
+// Copy one item (row block rb, groups g0, g0+1 if ng == 2) into a ring slot.
+__device__ __forceinline__ void issue_item(const GemvArgs& a, uint32_t slot, int rb, int g0, int ng, int lane) {
     const int nkb = a.in >> 6;
-    const uint4* src = a.qw + ((size_t)rb * nkb + 2 * g0) * 32 + lane;
+    const uint4* q = a.qw + ((size_t)rb * nkb + 2 * g0) * 32;
 #pragma unroll
-    for (int i = 0; i < kItemBlocks; ++i)
-        if (i < 2 * ng) it.w[i] = ldg_stream(src + i * 32);
-    const size_t mi = ((size_t)rb * a.G + g0) * 8 + (lane >> 2);
-#pragma unroll
-    for (int g = 0; g < kItemGroups; ++g) {
-        if (g < ng) {
-            it.s[g] = __ldg(a.sp + mi + 8 * g);
-            it.z[g] = __ldg(a.zp + mi + 8 * g);
-        }
+    for (int kb = 0; kb < 2 * kItemGroups; ++kb)
+        if (kb < 2 * ng) cp_async16(slot + kb * 512 + lane * 16, q + kb * 32 + lane);
+    if (lane < 2 * ng) cp_async16(slot + kItemQBytes + lane * 16, a.sp + ((size_t)rb * a.G + g0) * 8 + lane * 4);
+    if (lane == 31) {
+        const uint8_t* z = a.zp + ((size_t)rb * a.Gp + g0) * 8;
+        if (ng == 2) cp_async16(slot + kItemQBytes + kItemGroups * 32, z);
+        else cp_async8(slot + kItemQBytes + kItemGroups * 32, z);
     }
 }
 
@@ -105,32 +114,42 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     const int chunk = blockIdx.x, rt = blockIdx.y;
     const int g_begin = chunk * a.KC;
     const int g_end = min(a.G, g_begin + a.KC);
-    const int ncg = g_end - g_begin;                      // groups in this chunk
+    const int ncg = max(0, g_end - g_begin);
     const int nsub = (ncg + kItemGroups - 1) / kItemGroups;
     const int nrb = a.out >> 4;
     const int rb_begin = rt * a.RT;
     const int rb_end = min(nrb, rb_begin + a.RT);
-    const int nitems = max(0, rb_end - rb_begin) * nsub;
+    // this warp owns row blocks rb_begin + warp, + 8, ...; each over all subs of the chunk
+    const int my_rbs = (rb_end - rb_begin > warp) ? (rb_end - rb_begin - warp + kWarps - 1) / kWarps : 0;
+    const int nmine = my_rbs * nsub;
 
-    const int XS = a.KC * 128 + 16;                       // halves; row stride == 8 words mod 32
+    const int XS = a.KC * 128 + 16;                        // halves; row stride == 8 words mod 32
+    const int SR = a.RT * 16 + 4;                          // floats per token row of the partial tile
     __half* xs = reinterpret_cast<__half*>(smem);
-    const int RTR = a.RT * 16 + 4;                        // floats; == 4 words mod 32
-    float* red = reinterpret_cast<float*>(smem + (size_t)NT * 8 * XS * 2);
+    unsigned char* ring = smem + (size_t)NT * 8 * XS * 2;
+    float* red = reinterpret_cast<float*>(ring);          // reuses the ring once the stream is drained
+    const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kStages * kItemBytes);
+    const unsigned char* ring_p = ring + (size_t)warp * kStages * kItemBytes;
 
-    // ---- 1. first item's loads, zero the partial tile
-    Item cur, nxt;
-    int item = warp;
-    if (item < nitems) {
-        const int rb = rb_begin + item / nsub, sub = item % nsub;
-        const int g0 = g_begin + sub * kItemGroups;
-        load_item(cur, a, rb, g0, min(kItemGroups, g_end - g0), lane);
+    // producer cursor: (row block, sub) of the next item to copy, advanced incrementally
+    int p_rb = rb_begin + warp, p_sub = 0;
+    auto issue_next = [&](int stage) {
+        const int g0 = g_begin + p_sub * kItemGroups;
+        issue_item(a, ring_w + stage * kItemBytes, p_rb, g0, min(kItemGroups, g_end - g0), lane);
+        if (++p_sub == nsub) { p_sub = 0; p_rb += kWarps; }
+    };
+
+    // ---- weight stream prologue: first kStages-1 items in flight
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (s < nmine) issue_next(s);
+        cp_async_commit();
     }
-    for (int i = threadIdx.x; i < NT * 8 * RTR; i += kWarps * 32) red[i] = 0.f;
 
-    // ---- 2. wait for the rotation grid, stage X' chunk (zero rows >= T)
+    // ---- X' chunk (waits for the rotation grid)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
-        const int vec_per_row = ncg * 16;                  // 16-byte vectors per token row
+        const int vec_per_row = ncg * 16;
         const int total = NT * 8 * vec_per_row;
         for (int i = threadIdx.x; i < total; i += kWarps * 32) {
             const int tok = i / vec_per_row, v = i % vec_per_row;
@@ -142,126 +161,158 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     }
     __syncthreads();
 
-    // ---- 3. mainloop over this warp's items
+    // ---- mainloop: up to kMaxRbPerWarp row blocks, sums kept in registers
     const int gq = lane >> 2, qd = lane & 3;
-    for (; item < nitems; item += kWarps) {
-        const int rbl = item / nsub, sub = item % nsub;
-        const int g0 = g_begin + sub * kItemGroups;
-        const int ng = min(kItemGroups, g_end - g0);
-        const int nx = item + kWarps;
-        if (nx < nitems) {
-            const int rb2 = rb_begin + nx / nsub, sub2 = nx % nsub;
-            const int g2 = g_begin + sub2 * kItemGroups;
-            load_item(nxt, a, rb2, g2, min(kItemGroups, g_end - g2), lane);
-        }
-        // B fragment rows of this lane (token gq, gq + 8), at the item's first channel
-        const __half* xb[NT];
+    uint32_t xrow[NT];                                     // shared addresses of this lane's B rows
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) xb[nt] = xs + (size_t)(nt * 8 + gq) * XS + (g0 - g_begin) * 128 + 4 * qd;
-        float acc[NT][4];
+    for (int nt = 0; nt < NT; ++nt) xrow[nt] = smem_u32(xs + (size_t)(nt * 8 + gq) * XS + 4 * qd);
+    const uint32_t ring_s = smem_u32(ring_p);
+    float rsum[kMaxRbPerWarp][NT][4];
+    int i = 0, stage = 0, pstage = kStages - 1;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int r = 0; r < kMaxRbPerWarp; ++r) {
 #pragma unroll
-        for (int g = 0; g < kItemGroups; ++g) {
-            if (g < ng) {
-                // (q - z) is exact in fp16; s is applied to the group's fp32 partial sums
-                uint32_t zb0, zb1;
-                zero_bias(cur.z[g], zb0, zb1);
-                float p[NT][2][4];
+        for (int nt = 0; nt < NT; ++nt) rsum[r][nt][0] = rsum[r][nt][1] = rsum[r][nt][2] = rsum[r][nt][3] = 0.f;
+        if (r < my_rbs) {
+            float acc[NT][2][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) p[nt][c][0] = p[nt][c][1] = p[nt][c][2] = p[nt][c][3] = 0.f;
+                for (int c = 0; c < 2; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0.f;
+            for (int sub = 0; sub < nsub; ++sub, ++i) {
+                if (i + kStages - 1 < nmine) issue_next(pstage);
+                cp_async_commit();
+                pstage = (pstage + 1 == kStages) ? 0 : pstage + 1;
+                cp_async_wait<kStages - 1>();
+                __syncwarp();
+
+                const uint32_t slot = ring_s + stage * kItemBytes;
+                const int ng = min(kItemGroups, ncg - sub * kItemGroups);
+                const uint32_t kb_off = (uint32_t)(sub * kItemGroups * 128 * 2);   // bytes into the X' rows
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint4 wv = cur.w[2 * g + h];
-                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                for (int g = 0; g < kItemGroups; ++g) {
+                    if (g < ng) {
+                        uint32_t sc0, sc1;
+                        const Zero2 zc = zero_consts(lds8(slot + kItemQBytes + kItemGroups * 32 + g * 8 + gq));
+                        scale_pairs(lds32(slot + kItemQBytes + g * 32 + gq * 4), sc0, sc1);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t w = words[j];
-                        const uint32_t A[4] = {hsub2_rn(nib_pair_to_f16x2(w), zb0),
-                                               hsub2_rn(nib_pair_to_f16x2(w >> 8), zb1),
-                                               hsub2_rn(nib_pair_to_f16x2(w >> 4), zb0),
-                                               hsub2_rn(nib_pair_to_f16x2(w >> 12), zb1)};
-                        const int k = g * 128 + h * 64 + j * 16;
+                        for (int h = 0; h < 2; ++h) {
+                            const uint4 wv = lds128(slot + (2 * g + h) * 512 + lane * 16);
+                            const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            const uint2 bv = *reinterpret_cast<const uint2*>(xb[nt] + k);
-                            mma16816(p[nt][j & 1], A, bv.x, bv.y);
+                            for (int j = 0; j < 4; ++j) {
+                                uint32_t hh[4];
+                                dequant_word(words[j], zc, sc0, sc1, hh);
+                                const uint32_t A[4] = {hh[0], hh[2], hh[1], hh[3]};
+                                const uint32_t kbyte = kb_off + (uint32_t)((g * 128 + h * 64 + j * 16) * 2);
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    const uint2 bv = lds64(xrow[nt] + kbyte);
+                                    mma16816(acc[nt][j & 1], A, bv.x, bv.y);
+                                }
+                            }
                         }
                     }
                 }
-                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&cur.s[g]));
+                __syncwarp();                              // the slot may be refilled from here on
+                stage = (stage + 1 == kStages) ? 0 : stage + 1;
+            }
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    acc[nt][0] = fmaf(sf.x, p[nt][0][0] + p[nt][1][0], acc[nt][0]);
-                    acc[nt][1] = fmaf(sf.x, p[nt][0][1] + p[nt][1][1], acc[nt][1]);
-                    acc[nt][2] = fmaf(sf.y, p[nt][0][2] + p[nt][1][2], acc[nt][2]);
-                    acc[nt][3] = fmaf(sf.y, p[nt][0][3] + p[nt][1][3], acc[nt][3]);
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) rsum[r][nt][e] = acc[nt][0][e] + acc[nt][1][e];
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();                                       // every warp's stream drained: ring -> tile
+
+    // partial tile red[token][row] over this CTA's rows (rows of a warp: r*128 + warp*16 + ...)
+    for (int i2 = threadIdx.x; i2 < NT * 8 * SR; i2 += kWarps * 32) red[i2] = 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kMaxRbPerWarp; ++r) {
+        if (r < my_rbs) {
+            const int row = (warp + r * kWarps) * 16 + gq;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = nt * 8 + 2 * qd + e;
+                    red[t * SR + row] = rsum[r][nt][e];
+                    red[t * SR + row + 8] = rsum[r][nt][2 + e];
                 }
             }
         }
-        // partial sums -> shared tile red[token][row] (rows local to the CTA)
-        const int r0 = rbl * 16 + gq;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int t = nt * 8 + 2 * qd + e;
-                atomicAdd(red + t * RTR + r0, acc[nt][e]);
-                atomicAdd(red + t * RTR + r0 + 8, acc[nt][2 + e]);
-            }
-        }
-        cur = nxt;
     }
 
-    // ---- 4. split-k reduction across the cluster, fp16 store
-    const int nrows = max(0, rb_end - rb_begin) * 16;
+    // ---- split-k: CTA x of the cluster sums its share of the rows over all
+    // the cluster's tiles (distributed shared memory loads) and stores fp16
+    const int nrows_tile = max(0, rb_end - rb_begin) * 16;
     const int row0 = rb_begin * 16;
     if (a.nsplit == 1) {
         __syncthreads();
-        for (int i = threadIdx.x; i < a.T * nrows; i += kWarps * 32) {
-            const int t = i / nrows, r = i % nrows;
-            a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * RTR + r]);
+        for (int i = threadIdx.x; i < a.T * nrows_tile; i += kWarps * 32) {
+            const int t = i / nrows_tile, r = i % nrows_tile;
+            a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * SR + r]);
         }
         return;
     }
-    cluster_sync();                                        // all partial tiles complete
-    const int share = (nrows + a.nsplit - 1) / a.nsplit;
-    const int rlo = chunk * share, rhi = min(nrows, rlo + share);
-    const int n = max(0, rhi - rlo);
-    const uint32_t red_base = smem_u32(red);
+    cluster_sync();
+    const int rlo = chunk * a.share;
+    const int n = max(0, min(a.share, nrows_tile - rlo));
+    const uint32_t red_local = smem_u32(red);
     for (int i = threadIdx.x; i < a.T * n; i += kWarps * 32) {
         const int t = i / n, r = rlo + i % n;
-        const uint32_t off = red_base + (uint32_t)(t * RTR + r) * 4u;
+        const uint32_t off = red_local + (uint32_t)(t * SR + r) * 4u;
         float sum = 0.f;
-        for (int x = 0; x < a.nsplit; ++x) sum += ld_dsmem_f32(off, (uint32_t)x);
+        for (int x = 0; x < a.nsplit; ++x) sum += ld_dsmem(mapa(off, (uint32_t)x));
         a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(sum);
     }
-    cluster_sync();                                        // keep tiles alive until every reader is done
+    cluster_sync();                                        // tiles stay alive until every reader is done
 }
 
 struct GemvPlan {
-    int KC, nsplit, RT, rowtiles;
+    int KC, nsplit, RT, rowtiles, share;
     size_t smem;
 };
 
 static GemvPlan plan_gemv(int T, int64_t in, int64_t out, int sms) {
+    // Pick (k-chunk, row tile) minimising (waves x work per CTA): work is
+    // counted in (row block x group) units; two CTAs fit on an SM.
     const int G = (int)(in / 128);
     const int nrb = (int)(out / 16);
     const int NT = T > 8 ? 2 : 1;
-    GemvPlan p{};
-    const int kc_max = 20;
-    int nsplit = std::max(1, (G + kc_max - 1) / kc_max);
-    while (nsplit < 8 && (int64_t)nrb * nsplit < 4LL * sms && (G + nsplit) / (nsplit + 1) >= kItemGroups) ++nsplit;
-    nsplit = std::min(nsplit, 8);
-    p.KC = (G + nsplit - 1) / nsplit;
-    p.nsplit = (G + p.KC - 1) / p.KC;
-    const int want_tiles = std::max(1, (2 * sms + p.nsplit - 1) / p.nsplit);
-    p.RT = std::max(1, (nrb + want_tiles - 1) / want_tiles);
-    p.rowtiles = (nrb + p.RT - 1) / p.RT;
-    p.smem = (size_t)NT * 8 * (p.KC * 128 + 16) * 2 + (size_t)NT * 8 * (p.RT * 16 + 4) * 4;
-    return p;
+    const int kc_max = NT == 2 ? 10 : 20;                 // X' chunk <= ~41 KB
+    const int slots = 2 * sms;
+    GemvPlan best{};
+    double best_cost = 1e30;
+    for (int nsplit = 1; nsplit <= 16; ++nsplit) {
+        int KC = (G + nsplit - 1) / nsplit;
+        if (nsplit > 1) KC += KC & 1;
+        if (KC > kc_max) continue;
+        const int ns = (G + KC - 1) / KC;
+        if (ns != nsplit) continue;
+        for (int RT = 1; RT <= kWarps * kMaxRbPerWarp; ++RT) {
+            const int rowtiles = (nrb + RT - 1) / RT;
+            const int ctas = ns * rowtiles;
+            const int waves = (ctas + slots - 1) / slots;
+            const double per_warp = (double)((std::min(RT, nrb) + kWarps - 1) / kWarps) * KC;
+            // +2: pipeline fill per CTA; fewer CTAs than slots leaves SMs idle
+            const double cost = waves * (per_warp + 2.0) * (1.0 + 0.25 * (ctas < slots ? 1.0 - (double)ctas / slots : 0.0))
+                                + 0.02 * ns;
+            if (cost < best_cost - 1e-9) {
+                best_cost = cost;
+                best.KC = KC;
+                best.nsplit = ns;
+                best.RT = RT;
+                best.rowtiles = rowtiles;
+            }
+        }
+    }
+    best.share = 16 * ((best.RT + best.nsplit - 1) / best.nsplit);
+    best.smem = (size_t)NT * 8 * (best.KC * 128 + 16) * 2 +
+                std::max((size_t)NT * 8 * (best.RT * 16 + 4) * 4, (size_t)kWarps * kStages * kItemBytes);
+    return best;
 }
 
 template <int NT>
@@ -271,6 +322,8 @@ static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, bool pdl,
     cudaGetDevice(&dev);
     if (dev < 64 && !configured[dev]) {
         cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
@@ -317,9 +370,11 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.in = (int)in;
     a.out = (int)out;
     a.G = (int)(in / 128);
+    a.Gp = a.G + (a.G & 1);
     a.KC = p.KC;
     a.RT = p.RT;
     a.nsplit = p.nsplit;
+    a.share = p.share;
     a.qw = static_cast<const uint4*>(qw);
     a.sp = static_cast<const uint32_t*>(scp);
     a.zp = static_cast<const uint8_t*>(zp);

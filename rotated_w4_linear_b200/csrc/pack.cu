@@ -38,13 +38,16 @@ __global__ void pack_meta_kernel(const uint16_t* __restrict__ s, const uint8_t* 
                                  uint32_t* __restrict__ sp, uint8_t* __restrict__ zp, int G, int64_t n) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (rb, gi, g)
     if (i >= n) return;
+    const int Gp = G + (G & 1);
     const int g = (int)(i & 7);
     const int64_t rg = i >> 3;
     const int gi = (int)(rg % G);
     const int64_t rb = rg / G;
     const int64_t r0 = rb * 16 + g, r1 = r0 + 8;
     sp[i] = (uint32_t)s[r0 * G + gi] | ((uint32_t)s[r1 * G + gi] << 16);
-    zp[i] = (uint8_t)((z[r0 * G + gi] & 0xF) | ((z[r1 * G + gi] & 0xF) << 4));
+    const uint8_t zb = (uint8_t)((z[r0 * G + gi] & 0xF) | ((z[r1 * G + gi] & 0xF) << 4));
+    zp[(rb * Gp + gi) * 8 + g] = zb;
+    if ((G & 1) && gi == G - 1) zp[(rb * Gp + G) * 8 + g] = 0;   // padding group
 }
 
 cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out,
@@ -77,10 +80,11 @@ __global__ void dequant_kernel(const uint32_t* __restrict__ qw, const uint32_t* 
     const int g = lane >> 2, qd = lane & 3;
     const int gi = kb >> 1;
     const int64_t mi = (rb * G + gi) * 8 + g;
-    uint32_t zb0, zb1, sc0, sc1, h[4];
-    zero_bias(zp[mi], zb0, zb1);
+    const int Gp = G + (G & 1);
+    uint32_t sc0, sc1, h[4];
+    const Zero2 zc = zero_consts(zp[(rb * Gp + gi) * 8 + g]);
     scale_pairs(sp[mi], sc0, sc1);
-    dequant_word(qw[w], zb0, sc0, zb1, sc1, h);
+    dequant_word(qw[w], zc, sc0, sc1, h);
     const int k0 = kb * 64 + j * 16 + 4 * qd;
     __half* r0 = W + (rb * 16 + g) * (int64_t)in + k0;
     *reinterpret_cast<uint2*>(r0) = make_uint2(h[0], h[1]);

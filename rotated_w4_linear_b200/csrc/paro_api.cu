@@ -189,7 +189,8 @@ paro_status paro_pack_size(int64_t in, int64_t out, size_t* qb, size_t* sb, size
     if (!qb || !sb || !zb) return fail(PARO_ERR_ARG, "null size pointer");
     *qb = (size_t)(in * out / 2);
     *sb = (size_t)((out / 16) * (in / 128) * 8 * 4);
-    *zb = (size_t)((out / 16) * (in / 128) * 8);
+    const int64_t G = in / 128;
+    *zb = (size_t)((out / 16) * (G + (G & 1)) * 8);
     return PARO_OK;
 }
 

@@ -40,6 +40,7 @@ def test_pack_size(L):
     qb, sb, zb = binding.paro_pack_size(4096, 6144)
     assert qb == 4096 * 6144 // 2
     assert sb == 6144 // 16 * 32 * 8 * 4 and zb == 6144 // 16 * 32 * 8
+    assert binding.paro_pack_size(384, 48)[2] == 48 // 16 * 4 * 8       # 3 groups padded to 4
     # 0.5 + 2/128 + 0.5/128 bytes per weight
     assert (qb + sb + zb) / (4096 * 6144) == pytest.approx(0.5 + 2 / 128 + 0.5 / 128)
 

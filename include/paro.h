@@ -144,6 +144,12 @@ paro_status paro_linear(const paro_rot* rot, const void* X_dev,
                         void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,
                         void* workspace_dev, size_t workspace_bytes, paro_stream stream);
 
+/* Fault word of the current device: 0, or the code of a bounded wait inside a
+ * tensor-core kernel that ran out (about 2 s) because a pipeline stage never
+ * arrived; the kernel then abandoned its tile instead of hanging, and its
+ * output is not valid. Synchronous (copies one word); clear != 0 resets it. */
+paro_status paro_fault_status(int* code, int clear);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* paro_last_error(void);
 

@@ -34,6 +34,7 @@ _SIGS = {
     "paro_quantize_weights": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
     "paro_linear_workspace_size": [_i64, _i64, _i64, ctypes.POINTER(_sz)],
     "paro_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
+    "paro_fault_status": [ctypes.POINTER(_int), _int],
     "paro_last_error": [],
 }
 
@@ -121,6 +122,13 @@ def paro_rotate(rot: Rotation, X: torch.Tensor, Xr: Optional[torch.Tensor] = Non
         raise ValueError("X/Xr must be [tokens][in_features]")
     _check("paro_rotate", lib().paro_rotate(rot.handle, X.data_ptr(), Xr.data_ptr(), X.shape[0], _stream(stream)))
     return Xr
+
+
+def paro_fault_status(clear: bool = False) -> int:
+    """0, or the code of a bounded in-kernel wait that ran out (synchronous)."""
+    c = _int()
+    _check("paro_fault_status", lib().paro_fault_status(ctypes.byref(c), 1 if clear else 0))
+    return c.value
 
 
 def paro_pack_size(in_features: int, out_features: int):

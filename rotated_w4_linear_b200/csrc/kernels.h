@@ -32,4 +32,12 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
                         void* Y, int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes,
                         cudaStream_t s);
 
+// Prefill (tokens > 16): tcgen05 GEMM on X' (already rotated, in global memory),
+// launched as a programmatic dependent of the rotation kernel.
+cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, void* Y, int64_t T,
+                        int64_t in, int64_t out, cudaStream_t s);
+
+// Fault code left by a bounded wait that ran out (0 = none); optionally cleared.
+cudaError_t read_fault(unsigned int* code, bool clear);
+
 }  // namespace paro

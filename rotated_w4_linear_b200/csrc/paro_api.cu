@@ -65,6 +65,16 @@ extern "C" {
 
 const char* paro_last_error(void) { return g_err; }
 
+paro_status paro_fault_status(int* code, int clear) {
+    g_err[0] = 0;
+    if (!code) return fail(PARO_ERR_ARG, "code is null");
+    unsigned int c = 0;
+    cudaError_t e = paro::read_fault(&c, clear != 0);
+    if (e != cudaSuccess) return cuda_fail(e, "read fault word");
+    *code = (int)c;
+    return PARO_OK;
+}
+
 paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P, const int16_t* pairs,
                             const float* theta, const float* alpha) {
     g_err[0] = 0;
@@ -259,20 +269,15 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
         e = paro::launch_gemv(rd, X, qw, sp, zp, Y, T, in, out, ws, ws_bytes, s);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
-    // prefill: X' into the workspace, then the contraction over 16-token slices
+    // prefill: X' into the workspace, then the tensor-core GEMM
     const void* src = X;
     if (r) {
         e = paro::launch_rotate(r->dev, X, ws, T, s);
         if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
         src = ws;
     }
-    for (int64_t t0 = 0; t0 < T; t0 += 16) {
-        const int64_t n = (T - t0 < 16) ? (T - t0) : 16;
-        e = paro::launch_gemv(nullptr, static_cast<const char*>(src) + t0 * in * 2, qw, sp, zp,
-                              static_cast<char*>(Y) + t0 * out * 2, n, in, out, nullptr, 0, s);
-        if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
-    }
-    return PARO_OK;
+    e = paro::launch_gemm(src, qw, sp, zp, Y, T, in, out, s);
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "prefill launch");
 }
 
 }  // extern "C"

@@ -164,8 +164,10 @@ def _layer(B, in_f, out_f, K, P, seed, oracle_quant=True):
     (3, 384, 48, 8, 64),
     (8, 256, 80, 4, 13),
     (9, 384, 48, 1, 64),
-    (17, 512, 96, 8, 64),      # > 16 tokens: prefill path
-    (40, 384, 48, 8, 64),
+    (17, 512, 96, 8, 64),      # > 16 tokens: prefill path (tensor-core GEMM)
+    (40, 384, 48, 8, 64),      # partial 128-row tile, odd group count
+    (130, 512, 256, 8, 64),    # two 128-token tiles, ragged
+    (300, 256, 160, 4, 13),    # 256-token tiles, ragged rows and tokens
 ])
 def test_linear_parity_exhaustive(B, T, in_f, out_f, K, P):
     seed = synth.layer_seed(0, T * 7 + K)
@@ -177,6 +179,7 @@ def test_linear_parity_exhaustive(B, T, in_f, out_f, K, P):
     for _ in range(2):
         y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f, ws=ws))
         check_linear(y, x, pairs, theta, alpha, q, s, z)
+    assert B.paro_fault_status() == 0
 
 
 @pytest.mark.parametrize("T", [1, 5, 16])

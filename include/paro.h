@@ -144,6 +144,26 @@ paro_status paro_linear(const paro_rot* rot, const void* X_dev,
                         void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,
                         void* workspace_dev, size_t workspace_bytes, paro_stream stream);
 
+/* paro_linear for decode batches (tokens <= 16) that allocates nothing and
+ * takes no workspace: for callers that cannot allocate device memory, such
+ * as a serving engine that hands all device memory to its own pool at start-
+ * up, or code that must not call cudaMalloc while a CUDA graph is captured.
+ * No counterpart in the paper: this is a deployment convenience.
+ * The rotated activations X T^-1 go to a 1 MiB static device array that the
+ * library holds on every device that loads it until the process exits, so
+ * tokens * in_features * 2 must not exceed 1 MiB (else PARO_ERR_ARG; e.g. 16
+ * tokens x 32768 channels). Every call shares that array and it keeps the
+ * last call's contents (nothing in it needs clearing); calls that overlap on
+ * the GPU race on it, so serialise them (one stream, or events).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) once for that device; make that first call before
+ * any stream capture. Arguments are those of paro_linear without the
+ * workspace; the caller still owns X, the weights and Y. */
+paro_status paro_linear_noalloc(const paro_rot* rot, const void* X_dev,
+                                const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
+                                void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,
+                                paro_stream stream);
+
 /* Fault word of the current device: 0, or the code of a bounded wait inside a
  * tensor-core kernel that ran out (about 2 s) because a pipeline stage never
  * arrived; the kernel then abandoned its tile instead of hanging, and its

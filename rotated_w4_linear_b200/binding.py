@@ -34,6 +34,7 @@ _SIGS = {
     "paro_quantize_weights": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
     "paro_linear_workspace_size": [_i64, _i64, _i64, ctypes.POINTER(_sz)],
     "paro_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
+    "paro_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
     "paro_fault_status": [ctypes.POINTER(_int), _int],
     "paro_last_error": [],
 }
@@ -196,4 +197,18 @@ def paro_linear(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_featur
         _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"),
         _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
         _stream(stream)))
+    return Y
+
+
+def paro_linear_noalloc(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_features: int,
+                        Y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode (tokens <= 16) with the library's static scratch: no workspace,
+    no device allocation inside the call (Y is allocated here only if not given)."""
+    T, in_f = X.shape
+    if Y is None:
+        Y = torch.empty((T, out_features), dtype=torch.float16, device=X.device)
+    _check("paro_linear_noalloc", lib().paro_linear_noalloc(
+        rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
+        _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"),
+        _dev(Y, torch.float16, "Y"), T, in_f, out_features, _stream(stream)))
     return Y

@@ -384,4 +384,51 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Decode without any allocation by the caller or by the library.
+//
+// Some callers cannot allocate device memory for a workspace: a serving
+// engine that reserves all device memory for its own pool up front, or code
+// that must not call cudaMalloc while a CUDA graph is being captured. For
+// them the decode path can keep its only scratch (X T^-1, tokens x in fp16)
+// in this file-scope array instead. It lives on every device that loads the
+// library until the process exits. All calls share it and it keeps the last
+// call's contents (X T^-1 is fully written before it is read, so nothing needs
+// clearing); calls that overlap on the GPU race on it.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;   // 1 MiB: e.g. 16 tokens x 32768 channels
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device (in host
+// code the array's name is only a host-side stand-in, not a device address).
+cudaError_t noalloc_scratch(void** ptr) {
+    static void* addr[64] = {};
+    static bool ready[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!ready[dev]) {
+        e = cudaGetSymbolAddress(&addr[dev], g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        ready[dev] = true;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
+                                void* Y, int64_t T, int64_t in, int64_t out, cudaStream_t s) {
+    void* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    return launch_gemv(rot, X, qw, scp, zp, Y, T, in, out, scratch, kNoAllocScratchBytes, s);
+}
+
 }  // namespace paro

@@ -32,6 +32,11 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
                         void* Y, int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes,
                         cudaStream_t s);
 
+// Decode with the X' scratch in a static device array (no allocation anywhere).
+size_t noalloc_scratch_bytes();
+cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
+                                void* Y, int64_t T, int64_t in, int64_t out, cudaStream_t s);
+
 // Prefill (tokens > 16): tcgen05 GEMM on X' (already rotated, in global memory),
 // launched as a programmatic dependent of the rotation kernel.
 cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, void* Y, int64_t T,

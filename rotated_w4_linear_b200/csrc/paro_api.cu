@@ -65,6 +65,26 @@ extern "C" {
 
 const char* paro_last_error(void) { return g_err; }
 
+paro_status paro_linear_noalloc(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
+                                void* Y, int64_t T, int64_t in, int64_t out, paro_stream stream) {
+    g_err[0] = 0;
+    paro_status st = check_shape(in, out);
+    if (st != PARO_OK) return st;
+    if (T < 0) return fail(PARO_ERR_ARG, "tokens=%lld < 0", (long long)T);
+    if (T == 0) return PARO_OK;
+    if (T > 16) return fail(PARO_ERR_ARG, "tokens=%lld: this entry point serves decode batches of at most 16", (long long)T);
+    if ((size_t)T * (size_t)in * 2 > paro::noalloc_scratch_bytes())
+        return fail(PARO_ERR_ARG, "tokens x in_features x 2 = %zu bytes exceeds the %zu-byte static scratch",
+                    (size_t)T * (size_t)in * 2, paro::noalloc_scratch_bytes());
+    if (r && r->dev.in != in) return fail(PARO_ERR_ARG, "rotation prepared for in=%lld, layer has in=%lld", (long long)r->dev.in, (long long)in);
+    if (!X || !qw || !sp || !zp || !Y) return fail(PARO_ERR_ARG, "null pointer");
+    if (!aligned16(X) || !aligned16(qw) || !aligned16(sp) || !aligned16(zp) || !aligned16(Y))
+        return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
+    cudaError_t e = paro::launch_gemv_noalloc(r ? &r->dev : nullptr, X, qw, sp, zp, Y, T, in, out,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch (static scratch)");
+}
+
 paro_status paro_fault_status(int* code, int clear) {
     g_err[0] = 0;
     if (!code) return fail(PARO_ERR_ARG, "code is null");

@@ -228,6 +228,76 @@ def bench_rotate(args, torch, B, local):
     return 0
 
 
+# --------------------------------------------------------------------------- prefill
+def bench_prefill(args, torch, B, local):
+    """One Llama-3-8B-shaped layer's projections at --tokens: rotation +
+    tensor-core GEMM per projection, replayed as a CUDA graph. Reports the
+    GEMM FLOP rate (2 T in out per projection) against the measured dense
+    16-bit tensor peak, and the rotation overhead against the same GEMMs on
+    unrotated inputs (theta = 0, alpha = 1: no rotation launch)."""
+    torch.cuda.set_device(local)
+    T = args.tokens
+    dev = torch.device("cuda", local)
+    calls = []
+    for i, (name, n_in, n_out) in enumerate(PROJ):
+        seed = synth.layer_seed(3, i)
+        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
+        rot = B.paro_rot_create(pairs, theta, alpha)
+        w = torch.from_numpy(synth.weight(n_out, n_in, seed)).to(dev)
+        qw, sp, zp = B.paro_pack_weights(*B.paro_quantize_weights(rot, w))
+        del w
+        x = torch.from_numpy(synth.activations(T, n_in, seed)).to(dev)
+        calls.append(dict(rot=rot, n_in=n_in, n_out=n_out, qw=qw, sp=sp, zp=zp, x=x,
+                          y=torch.empty((T, n_out), dtype=torch.float16, device=dev),
+                          ws=B.workspace(T, n_in, n_out, dev)))
+
+    def step(rotate=True):
+        for p in calls:
+            B.paro_linear(p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
+                          Y=p["y"], ws=p["ws"])
+
+    step(); step(False)
+    torch.cuda.synchronize()
+    graphs = {}
+    for rot in (True, False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(rot)
+        graphs[rot] = g
+    for _ in range(args.warmup):
+        graphs[True].replay(); graphs[False].replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    times = {}
+    for rot in (True, False):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graphs[rot].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times[rot] = e0.elapsed_time(e1) / 1e3 / args.steps
+    flops = sum(2.0 * T * p["n_in"] * p["n_out"] for p in calls)
+    _, _, kind = peaks()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tc_peak = float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        tc_peak = 1400.0
+    tf = flops / times[False] / 1e12
+    print(json.dumps({"workload": f"prefill llama3-8b layer projections, {T} tokens, K={K_LAYERS}",
+                      "ms_per_layer": 1e3 * times[True], "ms_per_layer_unrotated": 1e3 * times[False],
+                      "TFLOP/s": flops / times[True] / 1e12, "TFLOP/s_gemm_only": tf,
+                      "rotation_overhead": times[True] / times[False] - 1.0,
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
+                                   "frac": tf / tc_peak, "peak_source": f"{kind} bf16_tflops_sustained "
+                                   "(fp16 and bf16 share the dense tensor rate)"}}), flush=True)
+    del graphs
+    for p in calls:
+        p["rot"].close()
+    return 0
+
+
 # --------------------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -238,8 +308,9 @@ def main():
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--impl", default="paro", choices=["paro", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "rotate"],
-                    help="decode: the headline step; rotate: paro_rotate alone (hidden 4096)")
+    ap.add_argument("--workload", default="decode", choices=["decode", "rotate", "prefill"],
+                    help="decode: the headline step; rotate: paro_rotate alone (hidden 4096); "
+                         "prefill: one layer's projections at --tokens (tensor-core GEMM)")
     ap.add_argument("--rot-k", type=int, default=8)
     ap.add_argument("--rot-pairs", type=int, default=64)
     args = ap.parse_args()
@@ -256,6 +327,8 @@ def main():
 
     if args.workload == "rotate":
         return bench_rotate(args, torch, B, local)
+    if args.workload == "prefill":
+        return bench_prefill(args, torch, B, local)
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -334,6 +407,26 @@ def main():
     elapsed = t_start.elapsed_time(t_end) / 1e3
     kern_s = k_start.elapsed_time(k_end) / 1e3
     clocks = clk.summary()
+
+    # per projection: the decode kernel alone, one graph per projection shape
+    per_proj = {}
+    for i, (name, n_in, n_out) in enumerate(PROJ):
+        sel = [p for p in calls if p["name"] == name]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for p in sel:
+                B.paro_linear(None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"], Y=p["y"], ws=p["ws"])
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (args.steps * len(sel))
+        nb = weight_bytes(n_in, n_out) + 2 * T * (n_in + n_out)
+        per_proj[name] = {"us": round(us, 2), "GB/s": round(nb / us / 1e3, 1)}
+        del g
     n_launch = args.steps * len(calls) * 2          # rotation + decode kernel per projection
     gemv_bytes = sum(weight_bytes(p["n_in"], p["n_out"]) + 2 * T * (p["n_in"] + p["n_out"]) for p in calls)
 
@@ -385,6 +478,7 @@ def main():
                      "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": {"value": step_bytes * args.steps * world / e2e_elapsed / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "decode_kernel_per_projection": per_proj,
         "gpu_launches": n_launch,
         "clocks": clocks,
     }

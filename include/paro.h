@@ -135,10 +135,12 @@ paro_status paro_linear_workspace_size(int64_t tokens, int64_t in_features, int6
  *                 initialisation needed); it receives X T^-1 in fp16. Calls
  *                 that share a workspace must not overlap on the GPU.
  * The rotation kernel writes X T^-1 into the workspace; the contraction runs
- * as a programmatic dependent launch of it (its weight loads start before
- * the rotation has finished). tokens <= 16 use the int4 decode kernel
- * (split-k reduced through distributed shared memory inside a thread-block
- * cluster); larger batches use the tensor-core prefill GEMM. */
+ * as a programmatic dependent launch of it (its weight loads start before the
+ * rotation has finished). tokens <= 16: the int4 decode kernel (warp MMAs fed
+ * by in-register dequantisation, split-k reduced through distributed shared
+ * memory inside a thread-block cluster); larger batches: the tensor-core
+ * GEMM (w_hat dequantised into tensor memory, X T^-1 tiles by TMA, 64/128/256
+ * tokens per tile). */
 paro_status paro_linear(const paro_rot* rot, const void* X_dev,
                         const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
                         void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,

@@ -25,6 +25,24 @@ __device__ __forceinline__ const uint8_t* rot_block(const uint8_t* rotp, int t, 
 }
 
 // ---------------------------------------------------------------------------
+// Exchange blocks for the rotation kernel, one per (layer t, group g), 1536 B:
+//   [32 lanes][uint4]: byte offsets (u16) in the warp's 512-byte exchange row
+//     where lane L stores its channels 4L..4L+3 (x: w0|w1<<16, y: w2|w3<<16)
+//     and where it loads their partners (z: r0|r1<<16, w: r2|r3<<16);
+//   [128 channels][float2]: (a, b) as in the rotation block.
+// The host chooses the positions so that each of the four stores and each of
+// the four loads of a warp hits 32 distinct banks: writes grouped by the slot
+// of the channel and reads grouped by the slot of its partner form a 4 x 4
+// bipartite multigraph with every node of degree 32, whose edges are coloured
+// with 32 colours (Koenig's theorem); the colour is the bank.
+// ---------------------------------------------------------------------------
+constexpr int kRotXBlockBytes = 32 * 16 + 128 * 8;
+
+__device__ __forceinline__ const uint8_t* rotx_block(const uint8_t* rotx, int t, int g, int G) {
+    return rotx + ((size_t)t * G + g) * kRotXBlockBytes;
+}
+
+// ---------------------------------------------------------------------------
 // int4 weight format (Kernel 4). For row block rb (16 output rows) and 64-wide
 // k block kb, 512 bytes: lane L (g = L >> 2, q = L & 3) owns 16 bytes = 4 words,
 // word j covering the 16x16 tile k in [64 kb + 16 j, +16). The word's nibbles:

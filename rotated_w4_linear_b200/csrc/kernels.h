@@ -12,6 +12,7 @@ struct RotDev {
     int K = 0;              // rotation layers
     int P = 0;              // active pairs per (layer, group)
     uint8_t* rotp = nullptr;       // [K][G] rotation blocks (fp32 coefficients)
+    uint8_t* rotx = nullptr;       // [K][G] exchange blocks: conflict-free positions + coefficients
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha
     uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
     double* alpha64 = nullptr;     // [in] alpha as fp64

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <new>
 #include <vector>
 
@@ -155,6 +156,44 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
             }
         }
     }
+    // exchange blocks: bank-conflict-free positions (edge colouring) + coefficients
+    std::vector<uint8_t> rotx((size_t)K * G * paro::kRotXBlockBytes);
+    for (int t = 0; t < K; ++t) {
+        for (int g = 0; g < G; ++g) {
+            const uint8_t* b = &rot32[((size_t)t * G + g) * paro::kRotBlockBytes];
+            const uint8_t* partner = b;
+            // buckets[i][j]: channels c with c % 4 == i (store slot) and partner % 4 == j (load slot)
+            std::vector<int> buckets[4][4];
+            for (int c = 0; c < 128; ++c) buckets[c & 3][partner[c] & 3].push_back(c);
+            int pos[128];
+            int used_rows[32] = {0};
+            for (int color = 0; color < 32; ++color) {
+                int perm[4] = {0, 1, 2, 3};
+                bool found = false;
+                do {
+                    bool ok = true;
+                    for (int i = 0; i < 4 && ok; ++i) ok = !buckets[i][perm[i]].empty();
+                    if (ok) { found = true; break; }
+                } while (std::next_permutation(perm, perm + 4));
+                if (!found) return fail(PARO_ERR_ARG, "internal: no conflict-free exchange layout");
+                for (int i = 0; i < 4; ++i) {
+                    const int c = buckets[i][perm[i]].back();
+                    buckets[i][perm[i]].pop_back();
+                    pos[c] = color + 32 * used_rows[color]++;
+                }
+            }
+            uint8_t* x = &rotx[((size_t)t * G + g) * paro::kRotXBlockBytes];
+            for (int l = 0; l < 32; ++l) {
+                uint16_t o[8];
+                for (int r = 0; r < 4; ++r) {
+                    o[r] = (uint16_t)(4 * pos[4 * l + r]);
+                    o[4 + r] = (uint16_t)(4 * pos[partner[4 * l + r]]);
+                }
+                memcpy(x + 16 * l, o, 16);
+            }
+            memcpy(x + 512, b + 128, 1024);
+        }
+    }
     std::vector<float> inv_alpha((size_t)in);
     std::vector<double> alpha64((size_t)in);
     for (int64_t c = 0; c < in; ++c) {
@@ -166,7 +205,8 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     const size_t o_inv = o_rot32 + round256(rot32.size());
     const size_t o_rot64 = o_inv + round256(inv_alpha.size() * sizeof(float));
     const size_t o_a64 = o_rot64 + round256(rot64.size());
-    const size_t total = o_a64 + round256(alpha64.size() * sizeof(double));
+    const size_t o_rotx = o_a64 + round256(alpha64.size() * sizeof(double));
+    const size_t total = o_rotx + round256(rotx.size());
 
     paro_rot* r = new (std::nothrow) paro_rot();
     if (!r) return fail(PARO_ERR_ARG, "out of host memory");
@@ -178,6 +218,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     if (e == cudaSuccess) e = cudaMemcpy(base + o_inv, inv_alpha.data(), inv_alpha.size() * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_rot64, rot64.data(), rot64.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !rotx.empty()) e = cudaMemcpy(base + o_rotx, rotx.data(), rotx.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { cudaFree(r->block); delete r; return cuda_fail(e, "cudaMemcpy(rotation tables)"); }
     r->dev.in = in;
     r->dev.G = G;
@@ -187,6 +228,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     r->dev.inv_alpha = reinterpret_cast<float*>(base + o_inv);
     r->dev.rotp64 = reinterpret_cast<uint8_t*>(base + o_rot64);
     r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);
+    r->dev.rotx = reinterpret_cast<uint8_t*>(base + o_rotx);
     *out = r;
     return PARO_OK;
 }
@@ -285,14 +327,15 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const paro::RotDev* rd = r ? &r->dev : nullptr;
     cudaError_t e;
-    if (T <= 16) {
+    if (T <= 16) {   // rotation + int4 decode kernel (programmatic dependent launch)
         e = paro::launch_gemv(rd, X, qw, sp, zp, Y, T, in, out, ws, ws_bytes, s);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
-    // prefill: X' into the workspace, then the tensor-core GEMM
+    // X' = X T^-1 into the workspace, then the tensor-core GEMM as a
+    // programmatic dependent launch
     const void* src = X;
-    if (r) {
-        e = paro::launch_rotate(r->dev, X, ws, T, s);
+    if (rd) {
+        e = paro::launch_rotate(*rd, X, ws, T, s);
         if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
         src = ws;
     }

@@ -6,8 +6,9 @@
 // Mapping: one warp owns one (group, token tile). Lane L holds channels
 // 4L..4L+3 of TT tokens, loaded as one 8-byte vector per token (a warp reads
 // 256 contiguous bytes per row). Partner values are exchanged through a
-// warp-private shared-memory slice each layer; rotation coefficients are read
-// from the prepared per-(layer, group) block (L1/L2 resident).
+// warp-private shared-memory row per token each layer, at positions chosen on
+// the host so that every store and load is bank-conflict-free; the next
+// layer's positions and coefficients are loaded while the current one runs.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -16,7 +17,7 @@ namespace paro {
 template <int TT>
 __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ X, __half* __restrict__ Xr,
                                                      int64_t T, int in, int G, int K,
-                                                     const uint8_t* __restrict__ rotp,
+                                                     const uint8_t* __restrict__ rotx,
                                                      const float* __restrict__ inv_alpha) {
     // a kernel launched after this one on the stream may start now; it waits
     // for this grid's completion before it reads Xr
@@ -43,39 +44,56 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
         v[i][3] = hi.y * ia.w;
     }
 
-    float(*b)[128] = buf[warp];
-    for (int tb = 0; tb < K; tb += 8) {
-        // all parameter loads of up to 8 layers are issued before any is used
-        uint32_t pw[8];
-        float4 c01[8], c23[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (tb + u < K) {
-                const uint8_t* blk = rot_block(rotp, tb + u, g, G);
-                pw[u] = __ldg(reinterpret_cast<const uint32_t*>(blk) + lane);
-                c01[u] = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane);
-                c23[u] = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane + 1);
-            }
+    // Each layer: every lane stores its 4 channels at the layer's positions
+    // in the warp's exchange rows (one 512-byte row per token), then loads
+    // the 4 partners; positions make every access bank-conflict-free.
+    float* row0 = &buf[warp][0][0];
+    uint4 off = make_uint4(0u, 0u, 0u, 0u);
+    float4 c01 = make_float4(1.f, 0.f, 1.f, 0.f), c23 = c01;
+    if (K > 0) {
+        const uint8_t* blk = rotx_block(rotx, 0, g, G);
+        off = __ldg(reinterpret_cast<const uint4*>(blk) + lane);
+        c01 = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane);
+        c23 = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane + 1);
+    }
+    for (int t = 0; t < K; ++t) {
+        uint4 off_n = off;
+        float4 c01_n = c01, c23_n = c23;
+        if (t + 1 < K) {                                   // next layer's parameters in flight
+            const uint8_t* blk = rotx_block(rotx, t + 1, g, G);
+            off_n = __ldg(reinterpret_cast<const uint4*>(blk) + lane);
+            c01_n = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane);
+            c23_n = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane + 1);
         }
+        // byte offsets -> float indices into the token-0 row; token i adds 128 i
+        float* w0 = row0 + ((off.x & 0xFFFFu) >> 2);
+        float* w1 = row0 + (off.x >> 18);
+        float* w2 = row0 + ((off.y & 0xFFFFu) >> 2);
+        float* w3 = row0 + (off.y >> 18);
+        const float* r0 = row0 + ((off.z & 0xFFFFu) >> 2);
+        const float* r1 = row0 + (off.z >> 18);
+        const float* r2 = row0 + ((off.w & 0xFFFFu) >> 2);
+        const float* r3 = row0 + (off.w >> 18);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (tb + u < K) {
-                const int p0 = pw[u] & 0xFF, p1 = (pw[u] >> 8) & 0xFF, p2 = (pw[u] >> 16) & 0xFF, p3 = pw[u] >> 24;
-#pragma unroll
-                for (int i = 0; i < TT; ++i)
-                    *reinterpret_cast<float4*>(&b[i][4 * lane]) = make_float4(v[i][0], v[i][1], v[i][2], v[i][3]);
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < TT; ++i) {
-                    const float q0 = b[i][p0], q1 = b[i][p1], q2 = b[i][p2], q3 = b[i][p3];
-                    v[i][0] = fmaf(c01[u].y, q0, c01[u].x * v[i][0]);
-                    v[i][1] = fmaf(c01[u].w, q1, c01[u].z * v[i][1]);
-                    v[i][2] = fmaf(c23[u].y, q2, c23[u].x * v[i][2]);
-                    v[i][3] = fmaf(c23[u].w, q3, c23[u].z * v[i][3]);
-                }
-                __syncwarp();
-            }
+        for (int i = 0; i < TT; ++i) {
+            w0[i * 128] = v[i][0];
+            w1[i * 128] = v[i][1];
+            w2[i * 128] = v[i][2];
+            w3[i * 128] = v[i][3];
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < TT; ++i) {
+            const float q0 = r0[i * 128], q1 = r1[i * 128], q2 = r2[i * 128], q3 = r3[i * 128];
+            v[i][0] = fmaf(c01.y, q0, c01.x * v[i][0]);
+            v[i][1] = fmaf(c01.w, q1, c01.z * v[i][1]);
+            v[i][2] = fmaf(c23.y, q2, c23.x * v[i][2]);
+            v[i][3] = fmaf(c23.w, q3, c23.z * v[i][3]);
+        }
+        __syncwarp();
+        off = off_n;
+        c01 = c01_n;
+        c23 = c23_n;
     }
 
 #pragma unroll
@@ -96,11 +114,11 @@ cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, c
     if (T <= 16) {   // decode batches: 4 tokens per warp for more warps in flight
         constexpr int TT = 4;
         const int64_t tasks = ((T + TT - 1) / TT) * r.G;
-        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotp, r.inv_alpha);
+        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotx, r.inv_alpha);
     } else {
         constexpr int TT = 8;
         const int64_t tasks = ((T + TT - 1) / TT) * r.G;
-        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotp, r.inv_alpha);
+        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotx, r.inv_alpha);
     }
     return cudaGetLastError();
 }

@@ -408,25 +408,30 @@ def main():
     kern_s = k_start.elapsed_time(k_end) / 1e3
     clocks = clk.summary()
 
-    # per projection: the decode kernel alone, one graph per projection shape
+    # per projection: the decode kernel alone, and rotation + decode kernel,
+    # one graph per projection shape
     per_proj = {}
     for i, (name, n_in, n_out) in enumerate(PROJ):
         sel = [p for p in calls if p["name"] == name]
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for p in sel:
-                B.paro_linear(None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"], Y=p["y"], ws=p["ws"])
-        g.replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
+        res = {}
+        for rotate in (False, True):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for p in sel:
+                    B.paro_linear(p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
+                                  Y=p["y"], ws=p["ws"])
             g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / (args.steps * len(sel))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            res[rotate] = e0.elapsed_time(e1) * 1e3 / (args.steps * len(sel))
+            del g
         nb = weight_bytes(n_in, n_out) + 2 * T * (n_in + n_out)
-        per_proj[name] = {"us": round(us, 2), "GB/s": round(nb / us / 1e3, 1)}
-        del g
+        per_proj[name] = {"us": round(res[False], 2), "GB/s": round(nb / res[False] / 1e3, 1),
+                          "us_with_rotation": round(res[True], 2)}
     n_launch = args.steps * len(calls) * 2          # rotation + decode kernel per projection
     gemv_bytes = sum(weight_bytes(p["n_in"], p["n_out"]) + 2 * T * (p["n_in"] + p["n_out"]) for p in calls)
 

@@ -43,6 +43,48 @@ __device__ __forceinline__ const uint8_t* rotx_block(const uint8_t* rotx, int t,
 }
 
 // ---------------------------------------------------------------------------
+// Quad exchange blocks for the decode rotation kernel, one per
+// (layer t, group g), 1280 B:
+//   [32 lanes][8 bytes]: float4-slot indices (0..127) in the warp's 2 KB
+//     exchange buffer where lane L stores channel 4L+j (bytes 0..3) and where
+//     it loads that channel's partner (bytes 4..7); a slot holds four tokens;
+//   [32 lanes][float4]: (a, b) of channels 4L and 4L+1, as in the rotation block;
+//   [32 lanes][float4]: (a, b) of channels 4L+2 and 4L+3.
+// A 16-byte shared access is served a quarter-warp (8 lanes) at a time; the
+// host gives the 8 lanes of every quarter distinct slots modulo 8 for each
+// store and each load (a proper 8-edge-colouring of the 16 x 16 bipartite
+// multigraph "store quarter-slot -> load quarter-slot", regular of degree
+// 8), so no access has a bank conflict.
+// ---------------------------------------------------------------------------
+constexpr int kRotQBlockBytes = 32 * 8 + 128 * 8;
+
+__device__ __forceinline__ const uint8_t* rotq_block(const uint8_t* rotq, int t, int g, int G) {
+    return rotq + ((size_t)t * G + g) * kRotQBlockBytes;
+}
+
+// Two fp32 lanes in one 64-bit register pair (sm_100 packed f32x2 arithmetic).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
 // int4 weight format (Kernel 4). For row block rb (16 output rows) and 64-wide
 // k block kb, 512 bytes: lane L (g = L >> 2, q = L & 3) owns 16 bytes = 4 words,
 // word j covering the 16x16 tile k in [64 kb + 16 j, +16). The word's nibbles:

@@ -4,30 +4,37 @@
 //
 // Launch: a grid of (nsplit, rowtiles) CTAs of 8 warps; CTAs with the same
 // row tile form one thread-block cluster along x, each owning a k-chunk of
-// KC 128-channel groups. The kernel is launched with programmatic stream
-// serialisation, so it starts while the rotation kernel still runs.
+// KC 128-channel groups. The kernel is a programmatic dependent launch: it
+// starts while the kernel before it still runs, streams its first weights,
+// and waits (griddepcontrol.wait) before it reads X'. It lets the next
+// kernel launch early in turn.
 //
-//   weight stream: warp w of a CTA owns the row blocks w, w + 8, ... of the
-//     tile, each over the whole k-chunk, as a sequence of items (16 rows x two
-//     groups: 2 KB of int4 codes + scales + zeros) streamed through a private
-//     3-stage shared-memory ring with cp.async (16-byte global->shared copies
-//     that bypass the registers): one commit group per item, wait on the
-//     oldest, so two items are in flight while one is consumed;
-//   X': after griddepcontrol.wait (the rotation grid has completed) the CTA
-//     copies its X' chunk (all tokens, zero rows >= T) into shared memory;
+//   work split: the CTA's items (one row block of 16 rows x two groups: 2 KB
+//     of int4 codes + scales + zeros) in row-block-major order are cut into
+//     eight equal contiguous runs, one per warp;
+//   weight stream: each warp streams its run through a private 3-stage
+//     shared-memory ring with cp.async (16-byte global->shared copies that
+//     bypass the registers): one commit group per item, wait on the oldest,
+//     so two items are in flight while one is consumed;
+//   X': the CTA copies its X' chunk (all tokens, zero rows >= T) into shared
+//     memory;
 //   math: each 32-bit int4 word is dequantised in registers (LOP3 into the
 //     1024 + q bit pattern, exact fp16 subtraction of 1024 + z, one rounded
 //     fp16 multiply: w_hat = fp16((q - z) s)) straight into an m16n8k16 A
 //     fragment; the B fragment (four consecutive channels of one token) comes
-//     from shared memory; fp32 accumulation in two independent chains;
-//   split-k: a row block's fp32 sums stay in registers over the chunk and
-//     are then stored into the CTA's shared tile [token][row]; after a
-//     cluster barrier CTA x sums its slice of the rows over the cluster's
-//     tiles with distributed shared memory loads and stores it as fp16. No
-//     global atomics, no workspace.
+//     from shared memory; fp32 accumulation in two independent chains, added
+//     into the CTA's partial tile [token][row] (shared-memory atomics) when
+//     the warp's run leaves a row block;
+//   split-k: after a cluster barrier CTA x sums its slice of the rows over
+//     the cluster's tiles with distributed shared memory loads and stores it
+//     as fp16. No global atomics, no workspace.
 // The k order inside each 16x16 tile follows the packed layout: the MMA's
 // logical k slot 2q+e holds channel 4q+e and slot 2q+8+e channel 4q+2+e.
 #include <algorithm>
+#include <cmath>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -41,7 +48,6 @@ constexpr int kStages = 3;
 constexpr int kItemGroups = 2;                            // groups per item
 constexpr int kItemQBytes = kItemGroups * 2 * 512;        // int4 codes
 constexpr int kItemBytes = kItemQBytes + kItemGroups * 32 + 16;   // + scales + zeros
-constexpr int kMaxRbPerWarp = 4;                          // row blocks a warp keeps sums for
 
 struct GemvArgs {
     const __half* Xr;     // [T][in] fp16, already rotated
@@ -109,6 +115,9 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, uint32_t slot, int
 
 template <int NT>
 __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) {
+    // the next kernel on the stream may launch now: it prefetches only its
+    // weights before it waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;");
     extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int chunk = blockIdx.x, rt = blockIdx.y;
@@ -118,141 +127,134 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     const int nsub = (ncg + kItemGroups - 1) / kItemGroups;
     const int nrb = a.out >> 4;
     const int rb_begin = rt * a.RT;
-    const int rb_end = min(nrb, rb_begin + a.RT);
-    // this warp owns row blocks rb_begin + warp, + 8, ...; each over all subs of the chunk
-    const int my_rbs = (rb_end - rb_begin > warp) ? (rb_end - rb_begin - warp + kWarps - 1) / kWarps : 0;
-    const int nmine = my_rbs * nsub;
+    const int nrbt = max(0, min(nrb, rb_begin + a.RT) - rb_begin);
+    // items (row block, sub) in row-block-major order; warp w takes the
+    // contiguous run [items*w/8, items*(w+1)/8)
+    const int items = nrbt * nsub;
+    const int i_lo = (int)(((int64_t)items * warp) / kWarps);
+    const int nmine = (int)(((int64_t)items * (warp + 1)) / kWarps) - i_lo;
 
     const int XS = a.KC * 128 + 16;                        // halves; row stride == 8 words mod 32
     const int SR = a.RT * 16 + 4;                          // floats per token row of the partial tile
     __half* xs = reinterpret_cast<__half*>(smem);
-    unsigned char* ring = smem + (size_t)NT * 8 * XS * 2;
-    float* red = reinterpret_cast<float*>(ring);          // reuses the ring once the stream is drained
+    float* red = reinterpret_cast<float*>(smem + (size_t)NT * 8 * XS * 2);
+    unsigned char* ring = reinterpret_cast<unsigned char*>(red + NT * 8 * SR);
     const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kStages * kItemBytes);
-    const unsigned char* ring_p = ring + (size_t)warp * kStages * kItemBytes;
 
-    // producer cursor: (row block, sub) of the next item to copy, advanced incrementally
-    int p_rb = rb_begin + warp, p_sub = 0;
+    // producer cursor: (row block, sub) of the next item to copy
+    int p_rb = rb_begin + (nsub ? i_lo / nsub : 0), p_sub = nsub ? i_lo % nsub : 0;
     auto issue_next = [&](int stage) {
         const int g0 = g_begin + p_sub * kItemGroups;
         issue_item(a, ring_w + stage * kItemBytes, p_rb, g0, min(kItemGroups, g_end - g0), lane);
-        if (++p_sub == nsub) { p_sub = 0; p_rb += kWarps; }
+        if (++p_sub == nsub) { p_sub = 0; ++p_rb; }
     };
 
-    // ---- weight stream prologue: first kStages-1 items in flight
+    // ---- weight stream prologue: first kStages-1 items in flight (weights
+    // are never written by the kernels this one may overlap)
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
         if (s < nmine) issue_next(s);
         cp_async_commit();
     }
 
-    // ---- X' chunk (waits for the rotation grid)
+    // ---- X' chunk and partial tile (waits for the previous grid: X' may be its output)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
         const int vec_per_row = ncg * 16;
         const int total = NT * 8 * vec_per_row;
         for (int i = threadIdx.x; i < total; i += kWarps * 32) {
-            const int tok = i / vec_per_row, v = i % vec_per_row;
+            const int tok = i / vec_per_row, v = i - tok * vec_per_row;
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
             if (tok < a.T)
                 val = __ldg(reinterpret_cast<const uint4*>(a.Xr + (size_t)tok * a.in + (size_t)g_begin * 128) + v);
             *reinterpret_cast<uint4*>(xs + (size_t)tok * XS + v * 8) = val;
         }
+        for (int i = threadIdx.x; i < NT * 8 * SR; i += kWarps * 32) red[i] = 0.f;
     }
     __syncthreads();
 
-    // ---- mainloop: up to kMaxRbPerWarp row blocks, sums kept in registers
+    // ---- mainloop: fp32 sums of the current row block in registers, added
+    // into the CTA's partial tile red[token][row] when the row block changes
     const int gq = lane >> 2, qd = lane & 3;
     uint32_t xrow[NT];                                     // shared addresses of this lane's B rows
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) xrow[nt] = smem_u32(xs + (size_t)(nt * 8 + gq) * XS + 4 * qd);
-    const uint32_t ring_s = smem_u32(ring_p);
-    float rsum[kMaxRbPerWarp][NT][4];
-    int i = 0, stage = 0, pstage = kStages - 1;
+    const uint32_t ring_s = smem_u32(ring) + (uint32_t)(warp * kStages * kItemBytes);
+    float acc[NT][2][4];
 #pragma unroll
-    for (int r = 0; r < kMaxRbPerWarp; ++r) {
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) rsum[r][nt][0] = rsum[r][nt][1] = rsum[r][nt][2] = rsum[r][nt][3] = 0.f;
-        if (r < my_rbs) {
-            float acc[NT][2][4];
+        for (int c = 0; c < 2; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0.f;
+    auto flush = [&](int rbl) {
+        float* base = red + rbl * 16 + gq;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0.f;
-            for (int sub = 0; sub < nsub; ++sub, ++i) {
-                if (i + kStages - 1 < nmine) issue_next(pstage);
-                cp_async_commit();
-                pstage = (pstage + 1 == kStages) ? 0 : pstage + 1;
-                cp_async_wait<kStages - 1>();
-                __syncwarp();
+            for (int e = 0; e < 2; ++e) {
+                const int t = nt * 8 + 2 * qd + e;
+                atomicAdd(base + t * SR, acc[nt][0][e] + acc[nt][1][e]);
+                atomicAdd(base + t * SR + 8, acc[nt][0][2 + e] + acc[nt][1][2 + e]);
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0.f;
+        }
+    };
+    int c_rbl = nsub ? i_lo / nsub : 0, c_sub = nsub ? i_lo % nsub : 0;   // item being consumed
+    int stage = 0, pstage = kStages - 1;
+    for (int i = 0; i < nmine; ++i) {
+        if (i + kStages - 1 < nmine) issue_next(pstage);
+        cp_async_commit();
+        pstage = (pstage + 1 == kStages) ? 0 : pstage + 1;
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
 
-                const uint32_t slot = ring_s + stage * kItemBytes;
-                const int ng = min(kItemGroups, ncg - sub * kItemGroups);
-                const uint32_t kb_off = (uint32_t)(sub * kItemGroups * 128 * 2);   // bytes into the X' rows
+        const uint32_t slot = ring_s + stage * kItemBytes;
+        const int ng = min(kItemGroups, ncg - c_sub * kItemGroups);
+        const uint32_t kb_off = (uint32_t)(c_sub * kItemGroups * 128 * 2);   // bytes into the X' rows
 #pragma unroll
-                for (int g = 0; g < kItemGroups; ++g) {
-                    if (g < ng) {
-                        uint32_t sc0, sc1;
-                        const Zero2 zc = zero_consts(lds8(slot + kItemQBytes + kItemGroups * 32 + g * 8 + gq));
-                        scale_pairs(lds32(slot + kItemQBytes + g * 32 + gq * 4), sc0, sc1);
+        for (int g = 0; g < kItemGroups; ++g) {
+            if (g < ng) {
+                uint32_t sc0, sc1;
+                const Zero2 zc = zero_consts(lds8(slot + kItemQBytes + kItemGroups * 32 + g * 8 + gq));
+                scale_pairs(lds32(slot + kItemQBytes + g * 32 + gq * 4), sc0, sc1);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint4 wv = lds128(slot + (2 * g + h) * 512 + lane * 16);
-                            const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                for (int h = 0; h < 2; ++h) {
+                    const uint4 wv = lds128(slot + (2 * g + h) * 512 + lane * 16);
+                    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                uint32_t hh[4];
-                                dequant_word(words[j], zc, sc0, sc1, hh);
-                                const uint32_t A[4] = {hh[0], hh[2], hh[1], hh[3]};
-                                const uint32_t kbyte = kb_off + (uint32_t)((g * 128 + h * 64 + j * 16) * 2);
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t hh[4];
+                        dequant_word(words[j], zc, sc0, sc1, hh);
+                        const uint32_t A[4] = {hh[0], hh[2], hh[1], hh[3]};
+                        const uint32_t kbyte = kb_off + (uint32_t)((g * 128 + h * 64 + j * 16) * 2);
 #pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    const uint2 bv = lds64(xrow[nt] + kbyte);
-                                    mma16816(acc[nt][j & 1], A, bv.x, bv.y);
-                                }
-                            }
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint2 bv = lds64(xrow[nt] + kbyte);
+                            mma16816(acc[nt][j & 1], A, bv.x, bv.y);
                         }
                     }
                 }
-                __syncwarp();                              // the slot may be refilled from here on
-                stage = (stage + 1 == kStages) ? 0 : stage + 1;
             }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) rsum[r][nt][e] = acc[nt][0][e] + acc[nt][1][e];
+        }
+        __syncwarp();                                      // the slot may be refilled from here on
+        stage = (stage + 1 == kStages) ? 0 : stage + 1;
+        if (++c_sub == nsub) {                             // row block done
+            flush(c_rbl);
+            c_sub = 0;
+            ++c_rbl;
         }
     }
+    if (nmine > 0 && c_sub != 0) flush(c_rbl);             // run ended inside a row block
     cp_async_wait<0>();
-    __syncthreads();                                       // every warp's stream drained: ring -> tile
-
-    // partial tile red[token][row] over this CTA's rows (rows of a warp: r*128 + warp*16 + ...)
-    for (int i2 = threadIdx.x; i2 < NT * 8 * SR; i2 += kWarps * 32) red[i2] = 0.f;
     __syncthreads();
-#pragma unroll
-    for (int r = 0; r < kMaxRbPerWarp; ++r) {
-        if (r < my_rbs) {
-            const int row = (warp + r * kWarps) * 16 + gq;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int t = nt * 8 + 2 * qd + e;
-                    red[t * SR + row] = rsum[r][nt][e];
-                    red[t * SR + row + 8] = rsum[r][nt][2 + e];
-                }
-            }
-        }
-    }
 
     // ---- split-k: CTA x of the cluster sums its share of the rows over all
     // the cluster's tiles (distributed shared memory loads) and stores fp16
-    const int nrows_tile = max(0, rb_end - rb_begin) * 16;
+    const int nrows_tile = nrbt * 16;
     const int row0 = rb_begin * 16;
     if (a.nsplit == 1) {
-        __syncthreads();
         for (int i = threadIdx.x; i < a.T * nrows_tile; i += kWarps * 32) {
-            const int t = i / nrows_tile, r = i % nrows_tile;
+            const int t = i / nrows_tile, r = i - t * nrows_tile;
             a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * SR + r]);
         }
         return;
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     const int n = max(0, min(a.share, nrows_tile - rlo));
     const uint32_t red_local = smem_u32(red);
     for (int i = threadIdx.x; i < a.T * n; i += kWarps * 32) {
-        const int t = i / n, r = rlo + i % n;
+        const int t = i / n, r = rlo + (i - t * n);
         const uint32_t off = red_local + (uint32_t)(t * SR + r) * 4u;
         float sum = 0.f;
         for (int x = 0; x < a.nsplit; ++x) sum += ld_dsmem(mapa(off, (uint32_t)x));
@@ -271,19 +273,65 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     cluster_sync();                                        // tiles stay alive until every reader is done
 }
 
+namespace {
+
 struct GemvPlan {
     int KC, nsplit, RT, rowtiles, share;
     size_t smem;
 };
 
-static GemvPlan plan_gemv(int T, int64_t in, int64_t out, int sms) {
-    // Pick (k-chunk, row tile) minimising (waves x work per CTA): work is
-    // counted in (row block x group) units; two CTAs fit on an SM.
+size_t gemv_smem(int NT, int KC, int RT) {
+    return (size_t)NT * 8 * (KC * 128 + 16) * 2 + (size_t)NT * 8 * (RT * 16 + 4) * 4 +
+           (size_t)kWarps * kStages * kItemBytes;
+}
+
+// CTAs of one launch that can be resident at once: clusters of `nsplit` CTAs
+// must sit inside one GPC, so for nsplit > 1 this is the driver's count of
+// co-resident clusters times nsplit (fewer than SMs x CTAs per SM).
+template <int NT>
+int gemv_slots(int dev, int nsplit, int per_sm) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, nsplit, per_sm);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int slots = sms * per_sm;
+    if (nsplit > 1 && cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                          cudaSuccess) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(nsplit, 1024, 1);
+        cfg.blockDim = dim3(kWarps * 32, 1, 1);
+        cfg.dynamicSmemBytes = per_sm >= 2 ? 100 * 1024 : 160 * 1024;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = nsplit;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int nc = 0;
+        if (cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
+                cudaSuccess &&
+            cudaOccupancyMaxActiveClusters(&nc, gemv_kernel<NT>, &cfg) == cudaSuccess && nc > 0)
+            slots = std::min(slots, nc * nsplit);
+        cudaGetLastError();   // a refused query leaves the SM-count estimate
+    }
+    cache[key] = slots;
+    return slots;
+}
+
+// Choose (k-chunk, row tile) for one shape: minimise waves x (items per warp
+// + pipeline fill), counting only CTAs that can be resident together.
+template <int NT>
+GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
     const int G = (int)(in / 128);
     const int nrb = (int)(out / 16);
-    const int NT = T > 8 ? 2 : 1;
     const int kc_max = NT == 2 ? 10 : 20;                 // X' chunk <= ~41 KB
-    const int slots = 2 * sms;
+    constexpr size_t kSmemPerSm = 228 * 1024, kReserved = 1024;
+    const size_t rot_reserve = K > 0 ? rotate_decode_smem(K, T) + kReserved : 0;
     GemvPlan best{};
     double best_cost = 1e30;
     for (int nsplit = 1; nsplit <= 16; ++nsplit) {
@@ -292,31 +340,49 @@ static GemvPlan plan_gemv(int T, int64_t in, int64_t out, int sms) {
         if (KC > kc_max) continue;
         const int ns = (G + KC - 1) / KC;
         if (ns != nsplit) continue;
-        for (int RT = 1; RT <= kWarps * kMaxRbPerWarp; ++RT) {
+        const int nsub = (KC + kItemGroups - 1) / kItemGroups;
+        for (int RT = 1; RT <= std::min(nrb, 64); ++RT) {
+            const size_t smem = gemv_smem(NT, KC, RT);
+            if (smem > 200 * 1024) break;
+            // two CTAs per SM, with room beside them for one CTA of the
+            // rotation kernel that runs before this one
+            const int per_sm = (2 * (smem + kReserved) + rot_reserve <= kSmemPerSm) ? 2 : 1;
+            const int slots = gemv_slots<NT>(dev, ns, per_sm);
             const int rowtiles = (nrb + RT - 1) / RT;
             const int ctas = ns * rowtiles;
             const int waves = (ctas + slots - 1) / slots;
-            const double per_warp = (double)((std::min(RT, nrb) + kWarps - 1) / kWarps) * KC;
-            // +2: pipeline fill per CTA; fewer CTAs than slots leaves SMs idle
-            const double cost = waves * (per_warp + 2.0) * (1.0 + 0.25 * (ctas < slots ? 1.0 - (double)ctas / slots : 0.0))
-                                + 0.02 * ns;
+            const double per_warp = std::ceil((double)RT * nsub / kWarps);
+            // +3: pipeline fill and epilogue per CTA; a partly empty wave
+            // still costs its share of HBM time
+            const double fill = (double)ctas / ((double)waves * slots);
+            const double cost = waves * (per_warp + 3.0) * (1.0 + 0.3 * (1.0 - fill)) + 0.05 * ns;
             if (cost < best_cost - 1e-9) {
                 best_cost = cost;
                 best.KC = KC;
                 best.nsplit = ns;
                 best.RT = RT;
                 best.rowtiles = rowtiles;
+                best.smem = smem;
             }
         }
     }
     best.share = 16 * ((best.RT + best.nsplit - 1) / best.nsplit);
-    best.smem = (size_t)NT * 8 * (best.KC * 128 + 16) * 2 +
-                std::max((size_t)NT * 8 * (best.RT * 16 + 4) * 4, (size_t)kWarps * kStages * kItemBytes);
     return best;
 }
 
 template <int NT>
-static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, bool pdl, cudaStream_t s) {
+GemvPlan cached_plan(int dev, int64_t in, int64_t out, int T, int K) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int64_t, int64_t, int, int>, GemvPlan> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, in, out, T, K);
+    auto it = cache.find(key);
+    if (it == cache.end()) it = cache.emplace(key, plan_gemv<NT>(dev, in, out, T, K)).first;
+    return it->second;
+}
+
+template <int NT>
+cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStream_t s) {
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -333,37 +399,37 @@ static cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, bool pdl,
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
-    int na = 0;
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = p.nsplit;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-    if (pdl) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.nsplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: the weight prologue overlaps the tail of
+    // the previous kernel; griddepcontrol.wait guards every read of X'
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = na;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, gemv_kernel<NT>, a);
 }
 
+}  // namespace
+
+// Decode: the rotation kernel writes X' = X T^-1 into ws (when rot is not
+// null), then the decode kernel runs on it; both are programmatic dependent
+// launches, so the decode kernel's weight stream starts during the rotation.
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
-                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, size_t /*ws_bytes*/,
-                        cudaStream_t s) {
+                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    int dev = 0, sms = 148;
+    int dev = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int K = rot ? rot->K : 0;
     const void* xr = X;
     if (rot) {
-        // X' = X T^-1 into the workspace; the GEMV waits on this grid in-kernel
-        cudaError_t e = launch_rotate(*rot, X, ws, T, s);
+        cudaError_t e = launch_rotate_decode(*rot, X, ws, T, s);
         if (e != cudaSuccess) return e;
         xr = ws;
     }
-    const GemvPlan p = plan_gemv((int)T, in, out, sms);
+    const GemvPlan p = (T > 8) ? cached_plan<2>(dev, in, out, (int)T, K) : cached_plan<1>(dev, in, out, (int)T, K);
     GemvArgs a{};
     a.Xr = static_cast<const __half*>(xr);
     a.T = (int)T;
@@ -379,7 +445,7 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.sp = static_cast<const uint32_t*>(scp);
     a.zp = static_cast<const uint8_t*>(zp);
     a.Y = static_cast<__half*>(Y);
-    cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, rot != nullptr, s) : launch_gemv_t<1>(a, p, rot != nullptr, s);
+    cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, s) : launch_gemv_t<1>(a, p, s);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -428,7 +494,7 @@ cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw
     void* scratch = nullptr;
     cudaError_t e = noalloc_scratch(&scratch);
     if (e != cudaSuccess) return e;
-    return launch_gemv(rot, X, qw, scp, zp, Y, T, in, out, scratch, kNoAllocScratchBytes, s);
+    return launch_gemv(rot, X, qw, scp, zp, Y, T, in, out, scratch, s);
 }
 
 }  // namespace paro

@@ -13,12 +13,17 @@ struct RotDev {
     int P = 0;              // active pairs per (layer, group)
     uint8_t* rotp = nullptr;       // [K][G] rotation blocks (fp32 coefficients)
     uint8_t* rotx = nullptr;       // [K][G] exchange blocks: conflict-free positions + coefficients
+    uint8_t* rotq = nullptr;       // [K][G] quad exchange blocks (decode prologue)
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha
     uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
     double* alpha64 = nullptr;     // [in] alpha as fp64
 };
 
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
+// Decode batches (1 <= T <= 16): one CTA per group, all layers' parameters in
+// shared memory; launched as a programmatic dependent of the previous kernel.
+cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
+size_t rotate_decode_smem(int K, int T);
 
 cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out,
                         void* qw, void* scp, void* zp, cudaStream_t s);
@@ -27,11 +32,10 @@ cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int6
 cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t* q, uint16_t* sc,
                             uint8_t* z, cudaStream_t s);
 
-// Decode path (tokens <= 16): rotation into ws (when rot is not null), then
-// the int4 GEMV launched as a programmatic dependent of it.
+// Decode path (tokens <= 16): the decode rotation kernel into ws (when rot
+// is not null), then the int4 decode kernel, both programmatic dependent launches.
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
-                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes,
-                        cudaStream_t s);
+                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s);
 
 // Decode with the X' scratch in a static device array (no allocation anywhere).
 size_t noalloc_scratch_bytes();

@@ -194,6 +194,61 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
             memcpy(x + 512, b + 128, 1024);
         }
     }
+    // quad exchange blocks: 16-byte slots, 8 lanes of a quarter-warp on 8 distinct
+    // slots mod 8 for every store and load (8 perfect matchings of an 8-regular
+    // bipartite multigraph, found one after another by augmenting paths)
+    std::vector<uint8_t> rotq((size_t)K * G * paro::kRotQBlockBytes);
+    for (int t = 0; t < K; ++t) {
+        for (int g = 0; g < G; ++g) {
+            const uint8_t* b = &rot32[((size_t)t * G + g) * paro::kRotBlockBytes];
+            const uint8_t* partner = b;
+            // channel c: store class (slot c%4, quarter of lane c/4), load class
+            // (slot, quarter) of the lane that owns its partner
+            int sc[128], lc[128], colour[128];
+            for (int c = 0; c < 128; ++c) {
+                sc[c] = (c & 3) * 4 + ((c >> 2) >> 3);
+                lc[c] = (partner[c] & 3) * 4 + ((partner[c] >> 2) >> 3);
+                colour[c] = -1;
+            }
+            for (int col = 0; col < 8; ++col) {
+                int match_r[16];                      // right class -> channel
+                for (int v = 0; v < 16; ++v) match_r[v] = -1;
+                bool vis[16];
+                // augmenting path from left class u over uncoloured channels
+                auto augment = [&](auto&& self, int u) -> bool {
+                    for (int c = 0; c < 128; ++c) {
+                        if (colour[c] >= 0 || sc[c] != u) continue;
+                        const int v = lc[c];
+                        if (vis[v]) continue;
+                        vis[v] = true;
+                        if (match_r[v] < 0 || self(self, sc[match_r[v]])) {
+                            match_r[v] = c;
+                            return true;
+                        }
+                    }
+                    return false;
+                };
+                for (int u = 0; u < 16; ++u) {
+                    for (int v = 0; v < 16; ++v) vis[v] = false;
+                    if (!augment(augment, u)) return fail(PARO_ERR_ARG, "internal: no conflict-free quad exchange layout");
+                }
+                for (int v = 0; v < 16; ++v) colour[match_r[v]] = col;
+            }
+            int pos[128], used[8] = {0};
+            for (int c = 0; c < 128; ++c) pos[c] = colour[c] + 8 * used[colour[c]]++;
+            uint8_t* x = &rotq[((size_t)t * G + g) * paro::kRotQBlockBytes];
+            for (int l = 0; l < 32; ++l) {
+                for (int j = 0; j < 4; ++j) {
+                    x[8 * l + j] = (uint8_t)pos[4 * l + j];
+                    x[8 * l + 4 + j] = (uint8_t)pos[partner[4 * l + j]];
+                }
+            }
+            for (int l = 0; l < 32; ++l) {   // (a, b) of channels 4l, 4l+1 | 4l+2, 4l+3
+                memcpy(x + 256 + 16 * l, b + 128 + 8 * (4 * l), 16);
+                memcpy(x + 768 + 16 * l, b + 128 + 8 * (4 * l + 2), 16);
+            }
+        }
+    }
     std::vector<float> inv_alpha((size_t)in);
     std::vector<double> alpha64((size_t)in);
     for (int64_t c = 0; c < in; ++c) {
@@ -206,7 +261,8 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     const size_t o_rot64 = o_inv + round256(inv_alpha.size() * sizeof(float));
     const size_t o_a64 = o_rot64 + round256(rot64.size());
     const size_t o_rotx = o_a64 + round256(alpha64.size() * sizeof(double));
-    const size_t total = o_rotx + round256(rotx.size());
+    const size_t o_rotq = o_rotx + round256(rotx.size());
+    const size_t total = o_rotq + round256(rotq.size());
 
     paro_rot* r = new (std::nothrow) paro_rot();
     if (!r) return fail(PARO_ERR_ARG, "out of host memory");
@@ -219,6 +275,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     if (e == cudaSuccess) e = cudaMemcpy(base + o_rot64, rot64.data(), rot64.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !rotx.empty()) e = cudaMemcpy(base + o_rotx, rotx.data(), rotx.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !rotq.empty()) e = cudaMemcpy(base + o_rotq, rotq.data(), rotq.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { cudaFree(r->block); delete r; return cuda_fail(e, "cudaMemcpy(rotation tables)"); }
     r->dev.in = in;
     r->dev.G = G;
@@ -229,6 +286,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     r->dev.rotp64 = reinterpret_cast<uint8_t*>(base + o_rot64);
     r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);
     r->dev.rotx = reinterpret_cast<uint8_t*>(base + o_rotx);
+    r->dev.rotq = reinterpret_cast<uint8_t*>(base + o_rotq);
     *out = r;
     return PARO_OK;
 }
@@ -327,8 +385,8 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const paro::RotDev* rd = r ? &r->dev : nullptr;
     cudaError_t e;
-    if (T <= 16) {   // rotation + int4 decode kernel (programmatic dependent launch)
-        e = paro::launch_gemv(rd, X, qw, sp, zp, Y, T, in, out, ws, ws_bytes, s);
+    if (T <= 16) {   // decode rotation kernel into ws, then the int4 decode kernel
+        e = paro::launch_gemv(rd, X, qw, sp, zp, Y, T, in, out, ws, s);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
     // X' = X T^-1 into the workspace, then the tensor-core GEMM as a

@@ -22,6 +22,9 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
     // a kernel launched after this one on the stream may start now; it waits
     // for this grid's completion before it reads Xr
     asm volatile("griddepcontrol.launch_dependents;");
+    // this kernel is itself a programmatic dependent launch: X may be the
+    // output of the kernel before it, so X is read only after this wait
+    // (the rotation parameters are never written by a kernel on the path)
     __shared__ __align__(16) float buf[4][TT][128];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t task = (int64_t)blockIdx.x * 4 + warp;
@@ -31,6 +34,7 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
     const int c0 = g * 128 + 4 * lane;
 
     const float4 ia = __ldg(reinterpret_cast<const float4*>(inv_alpha + c0));
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     float v[TT][4];
 #pragma unroll
     for (int i = 0; i < TT; ++i) {
@@ -107,20 +111,152 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
     }
 }
 
+// Decode batches (tokens <= 16): one CTA per 128-channel group, warp q
+// rotates tokens 4q..4q+3. All K layers' quad exchange blocks of the group
+// are copied into shared memory before the wait for the previous grid (they
+// are never written by a kernel on the path), so the layers run from shared
+// memory: lane L holds channels 4L..4L+3 of four tokens, exchanges partner
+// values as float4 slots (conflict-free), and updates two tokens per packed
+// f32x2 multiply and fma, the same operations in the same order as
+// rotate_kernel, so X' is bit-identical.
+__global__ void __launch_bounds__(128) rotate_decode_kernel(const __half* __restrict__ X, __half* __restrict__ Xr,
+                                                            int T, int in, int G, int K,
+                                                            const uint8_t* __restrict__ rotq,
+                                                            const float* __restrict__ inv_alpha) {
+    asm volatile("griddepcontrol.launch_dependents;");
+    extern __shared__ __align__(16) unsigned char sm[];
+    const int lane = threadIdx.x & 31, q = threadIdx.x >> 5;
+    const int g = blockIdx.x;
+    unsigned char* prm = sm;                               // [K][kRotQBlockBytes]
+    const uint32_t xbuf = (uint32_t)__cvta_generic_to_shared(sm + (size_t)K * kRotQBlockBytes) + q * 2048u;
+    {
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(prm);
+        const int per_layer = kRotQBlockBytes / 16;
+        for (int i = threadIdx.x; i < K * per_layer; i += blockDim.x) {
+            const int t = i / per_layer, v = i - t * per_layer;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16u * i),
+                         "l"(rotq_block(rotq, t, g, G) + 16 * v) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const int c0 = g * 128 + 4 * lane;
+    const float4 ia = __ldg(reinterpret_cast<const float4*>(inv_alpha + c0));
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // X may be the previous grid's output
+    uint64_t v[4][2];                                      // [channel j][token pair]
+    {
+        float x[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * q + i;
+            uint2 raw = make_uint2(0u, 0u);
+            if (t < T) raw = __ldg(reinterpret_cast<const uint2*>(X + (size_t)t * in + c0));
+            const float2 lo = __half22float2(*reinterpret_cast<__half2*>(&raw.x));
+            const float2 hi = __half22float2(*reinterpret_cast<__half2*>(&raw.y));
+            x[i][0] = lo.x * ia.x;
+            x[i][1] = lo.y * ia.y;
+            x[i][2] = hi.x * ia.z;
+            x[i][3] = hi.y * ia.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[j][0] = f2_pack(x[0][j], x[1][j]);
+            v[j][1] = f2_pack(x[2][j], x[3][j]);
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    for (int t = 0; t < K; ++t) {
+        const unsigned char* blk = prm + (size_t)t * kRotQBlockBytes;
+        const uint2 pos = *reinterpret_cast<const uint2*>(blk + 8 * lane);
+        const float4 c01 = *reinterpret_cast<const float4*>(blk + 256 + 16 * lane);
+        const float4 c23 = *reinterpret_cast<const float4*>(blk + 768 + 16 * lane);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t slot = (pos.x >> (8 * j)) & 0xFFu;
+            asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(xbuf + 16u * slot), "l"(v[j][0]), "l"(v[j][1])
+                         : "memory");
+        }
+        __syncwarp();
+        uint64_t p[4][2];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t slot = (pos.y >> (8 * j)) & 0xFFu;
+            asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(p[j][0]), "=l"(p[j][1]) : "r"(xbuf + 16u * slot)
+                         : "memory");
+        }
+        __syncwarp();
+        const float ca[4] = {c01.x, c01.z, c23.x, c23.z}, cb[4] = {c01.y, c01.w, c23.y, c23.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint64_t a2 = f2_pack(ca[j], ca[j]), b2 = f2_pack(cb[j], cb[j]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) v[j][h] = f2_fma(b2, p[j][h], f2_mul(a2, v[j][h]));
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float2 w0 = f2_unpack(v[0][h]), w1 = f2_unpack(v[1][h]);
+        const float2 w2 = f2_unpack(v[2][h]), w3 = f2_unpack(v[3][h]);
+        const int t = 4 * q + 2 * h;
+        if (t < T)
+            *reinterpret_cast<uint2*>(Xr + (size_t)t * in + c0) =
+                make_uint2(pack_half2(w0.x, w1.x), pack_half2(w2.x, w3.x));
+        if (t + 1 < T)
+            *reinterpret_cast<uint2*>(Xr + (size_t)(t + 1) * in + c0) =
+                make_uint2(pack_half2(w0.y, w1.y), pack_half2(w2.y, w3.y));
+    }
+}
+
+size_t rotate_decode_smem(int K, int T) { return (size_t)K * kRotQBlockBytes + (size_t)((T + 3) / 4) * 2048; }
+
+cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    if (T > 16) return cudaErrorInvalidValue;
+    const size_t smem = rotate_decode_smem(r.K, (int)T);
+    if (smem > 48 * 1024) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(rotate_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)r.G, 1, 1);
+    cfg.blockDim = dim3((unsigned)(32 * ((T + 3) / 4)), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_decode_kernel, static_cast<const __half*>(X),
+                                             static_cast<__half*>(Xr), (int)T, (int)r.in, r.G, r.K,
+                                             (const uint8_t*)r.rotq, (const float*)r.inv_alpha);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int TT>
+static cudaError_t launch_rotate_t(const RotDev& r, const __half* x, __half* y, int64_t T, cudaStream_t s) {
+    const int64_t tasks = ((T + TT - 1) / TT) * r.G;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((tasks + 3) / 4), 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, rotate_kernel<TT>, x, y, T, (int)r.in, r.G, r.K, (const uint8_t*)r.rotx,
+                              (const float*)r.inv_alpha);
+}
+
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     const __half* x = static_cast<const __half*>(X);
     __half* y = static_cast<__half*>(Xr);
-    if (T <= 16) {   // decode batches: 4 tokens per warp for more warps in flight
-        constexpr int TT = 4;
-        const int64_t tasks = ((T + TT - 1) / TT) * r.G;
-        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotx, r.inv_alpha);
-    } else {
-        constexpr int TT = 8;
-        const int64_t tasks = ((T + TT - 1) / TT) * r.G;
-        rotate_kernel<TT><<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(x, y, T, (int)r.in, r.G, r.K, r.rotx, r.inv_alpha);
-    }
-    return cudaGetLastError();
+    if (T <= 16) return launch_rotate_decode(r, X, Xr, T, s);
+    const cudaError_t e = launch_rotate_t<8>(r, x, y, T, s);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace paro

@@ -86,6 +86,22 @@ def test_rotate_parity(B, T, in_f, K, P):
     check_rotation(got, x, pairs, theta, alpha)
 
 
+@pytest.mark.parametrize("in_f,K,P", [(4096, 8, 64), (14336, 16, 13), (384, 3, 64)])
+def test_rotate_decode_kernel_matches_general_kernel(B, in_f, K, P):
+    """Batches of at most 16 tokens take the decode rotation kernel (float4
+    exchange, packed f32x2 arithmetic); larger batches the general one. Both
+    apply the same operations in the same order: identical bits."""
+    seed = synth.layer_seed(1, 77 + K)
+    pairs, theta, alpha = synth.rotation_params(in_f, K, seed, pairs_per_group=P)
+    x = synth.activations(24, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    big = host(B.paro_rotate(rot, dev(x)))
+    for T in (1, 7, 16):
+        small = host(B.paro_rotate(rot, dev(x[:T])))
+        assert np.array_equal(small.view(np.uint16), big[:T].view(np.uint16)), T
+    check_rotation(big[:16], x[:16], pairs, theta, alpha)
+
+
 @pytest.mark.parametrize("T", [2048, 8192])
 def test_rotate_full_size_sampled_rows(B, T):
     seed = synth.layer_seed(1, T)

@@ -113,6 +113,50 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(dist, values, device=None):
+    """Every rank passes its own device times; every rank gets the maximum of
+    each over all ranks (the slowest rank defines the step)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_bytes, n_calls,
+                hbm_peak, peak_kind, h2d, d2h, per_proj, n_launch, clocks):
+    """The JSON line of the decode workload. Times are max-over-ranks seconds
+    for args.steps steps; every rank moved step_bytes per step."""
+    value = step_bytes * args.steps * world / elapsed / 1e9
+    achieved = gemv_bytes * args.steps / kern_s / 1e9
+    return {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 (int4 weights, fp32 accumulate)",
+        "data": "synthetic (seeded Llama-3-8B-shaped layers; weights quantised on the GPU from T W)",
+        "config": config(args),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "gemv_kernel (int4 decode)",
+                     "us_per_launch": 1e6 * kern_s / (args.steps * n_calls),
+                     "peak_source": f"{peak_kind} hbm_gbs"},
+        "e2e": {"value": step_bytes * args.steps * world / e2e_elapsed / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "decode_kernel_per_projection": per_proj,
+        "gpu_launches": n_launch,
+        "clocks": clocks,
+    }
+
+
+def emit(line, rank):
+    """Rank 0 prints the one JSON line; the other ranks print nothing."""
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+        return True
+    return False
+
+
 # --------------------------------------------------------------------------- oracle baseline
 def cpu_baseline(tokens: int, budget_s: float = 12.0):
     """The CPU fp64 oracle as it stands, on a bounded sample: whole projections
@@ -463,34 +507,12 @@ def main():
     torch.cuda.synchronize()
     e2e_elapsed = e0.elapsed_time(e1) / 1e3
 
-    if dist:
-        t = torch.tensor([elapsed, e2e_elapsed, kern_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed, e2e_elapsed, kern_s = (float(v) for v in t.tolist())
-
-    total_bytes = step_bytes * args.steps * world
-    value = total_bytes / elapsed / 1e9
-    achieved = gemv_bytes * args.steps / kern_s / 1e9
-    line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16 (int4 weights, fp32 accumulate)",
-        "data": "synthetic (seeded Llama-3-8B-shaped layers; weights quantised on the GPU from T W)",
-        "config": config(args),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "gemv_kernel (int4 decode)",
-                     "us_per_launch": 1e6 * kern_s / (args.steps * len(calls)),
-                     "peak_source": f"{peak_kind} hbm_gbs"},
-        "e2e": {"value": step_bytes * args.steps * world / e2e_elapsed / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "decode_kernel_per_projection": per_proj,
-        "gpu_launches": n_launch,
-        "clocks": clocks,
-    }
+    elapsed, e2e_elapsed, kern_s = max_over_ranks(dist, [elapsed, e2e_elapsed, kern_s], dev)
+    line = decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_bytes, len(calls),
+                       hbm_peak, peak_kind, h2d, d2h, per_proj, n_launch, clocks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    emit(line, rank)
     del g_step, g_gemv
     for projs in layers:
         for p in projs:

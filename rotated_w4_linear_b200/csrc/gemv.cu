@@ -62,8 +62,10 @@ struct GemvArgs {
     __half* Y;
 };
 
+// Not volatile: the MMA reads registers only, so the compiler may schedule
+// it freely against the shared-memory loads and the dequantisation.
 __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -176,10 +178,14 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     // ---- mainloop: fp32 sums of the current row block in registers, added
     // into the CTA's partial tile red[token][row] when the row block changes
     const int gq = lane >> 2, qd = lane & 3;
-    uint32_t xrow[NT];                                     // shared addresses of this lane's B rows
+    // Shared memory is read through plain C++ loads (not asm), so the compiler
+    // sees them as memory accesses: it can hoist them for latency but not
+    // across the cp.async waits and warp barriers that order the ring.
+    const unsigned char* xrow[NT];                         // this lane's B rows
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) xrow[nt] = smem_u32(xs + (size_t)(nt * 8 + gq) * XS + 4 * qd);
-    const uint32_t ring_s = smem_u32(ring) + (uint32_t)(warp * kStages * kItemBytes);
+    for (int nt = 0; nt < NT; ++nt)
+        xrow[nt] = reinterpret_cast<const unsigned char*>(xs + (size_t)(nt * 8 + gq) * XS + 4 * qd);
+    const unsigned char* ring_p = ring + (size_t)warp * kStages * kItemBytes;
     float acc[NT][2][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -208,28 +214,28 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
         cp_async_wait<kStages - 1>();
         __syncwarp();
 
-        const uint32_t slot = ring_s + stage * kItemBytes;
+        const unsigned char* slot = ring_p + stage * kItemBytes;
         const int ng = min(kItemGroups, ncg - c_sub * kItemGroups);
-        const uint32_t kb_off = (uint32_t)(c_sub * kItemGroups * 128 * 2);   // bytes into the X' rows
+        const int kb_off = c_sub * kItemGroups * 128 * 2;  // bytes into the X' rows
 #pragma unroll
         for (int g = 0; g < kItemGroups; ++g) {
             if (g < ng) {
                 uint32_t sc0, sc1;
-                const Zero2 zc = zero_consts(lds8(slot + kItemQBytes + kItemGroups * 32 + g * 8 + gq));
-                scale_pairs(lds32(slot + kItemQBytes + g * 32 + gq * 4), sc0, sc1);
+                const Zero2 zc = zero_consts(slot[kItemQBytes + kItemGroups * 32 + g * 8 + gq]);
+                scale_pairs(*reinterpret_cast<const uint32_t*>(slot + kItemQBytes + g * 32 + gq * 4), sc0, sc1);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const uint4 wv = lds128(slot + (2 * g + h) * 512 + lane * 16);
+                    const uint4 wv = *reinterpret_cast<const uint4*>(slot + (2 * g + h) * 512 + lane * 16);
                     const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t hh[4];
                         dequant_word(words[j], zc, sc0, sc1, hh);
                         const uint32_t A[4] = {hh[0], hh[2], hh[1], hh[3]};
-                        const uint32_t kbyte = kb_off + (uint32_t)((g * 128 + h * 64 + j * 16) * 2);
+                        const int kbyte = kb_off + (g * 128 + h * 64 + j * 16) * 2;
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            const uint2 bv = lds64(xrow[nt] + kbyte);
+                            const uint2 bv = *reinterpret_cast<const uint2*>(xrow[nt] + kbyte);
                             mma16816(acc[nt][j & 1], A, bv.x, bv.y);
                         }
                     }

@@ -1,0 +1,64 @@
+"""Host logic of bench.py's multi-GPU path, run as two gloo ranks on the CPU.
+
+Every rank times its own replicas; the step time is the maximum over ranks,
+`value` counts the bytes of all ranks, and only rank 0 prints the JSON line.
+"""
+import json
+import os
+import socket
+import sys
+import types
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, outdir):
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r is slower on one timer and faster on another
+        mine = [1.0 + rank, 2.0 - rank, 0.5 + 0.25 * rank]
+        got = bench.max_over_ranks(dist, mine)
+        args = types.SimpleNamespace(steps=10, warmup=3, tokens=16, layers=4, gpus=world)
+        line = bench.decode_line(args, world, got[0], got[1], got[2], step_bytes=1e9, gemv_bytes=5e8,
+                                 n_calls=16, hbm_peak=6454.9, peak_kind="measured", h2d=1, d2h=2,
+                                 per_proj={}, n_launch=320, clocks={})
+        printed = bench.emit(line, rank)
+        with open(os.path.join(outdir, f"rank{rank}.json"), "w") as f:
+            json.dump({"got": got, "line": line, "printed": printed}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_time_and_single_line(tmp_path):
+    world = 2
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    for r in res:
+        assert r["got"] == [2.0, 2.0, 0.75]                 # element-wise max over ranks
+    assert [r["printed"] for r in res] == [True, False]     # one JSON line, from rank 0
+    line = res[0]["line"]
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak"
+    assert line["value"] == pytest.approx(1e9 * 10 * 2 / 2.0 / 1e9)   # all ranks' bytes / slowest time
+    assert line["ms_per_step"] == pytest.approx(1e3 * 2.0 / 10)
+    assert line["roofline"]["achieved"] == pytest.approx(5e8 * 10 / 0.75 / 1e9)   # per-rank kernel rate
+    assert line["e2e"]["value"] == pytest.approx(1e9 * 10 * 2 / 2.0 / 1e9)
+
+
+def test_single_process_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(None, [3, 1.5]) == [3.0, 1.5]

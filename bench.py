@@ -51,6 +51,13 @@ def call_bytes(T, n_in, n_out):
     return weight_bytes(n_in, n_out) + 2 * T * n_in + 2 * T * n_out + rot_param_bytes(n_in)
 
 
+# DRAM bytes (read + write) per decode-kernel launch, mean over the four
+# projections (qkv 13.24 MB, o 8.88 MB, gate+up 61.18 MB, down 30.99 MB), from
+# one ncu capture of the current kernel at 16 tokens; the command is in
+# profiles/gemv_kernel_gate_up_4096x28672_t16.md. None once the kernel changes.
+GEMV_TRAFFIC_PER_LAUNCH_T16 = (13238016 + 8875264 + 61180672 + 30993920) / 4
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -138,7 +145,9 @@ def decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_byte
         "data": "synthetic (seeded Llama-3-8B-shaped layers; weights quantised on the GPU from T W)",
         "config": config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "gemv_kernel (int4 decode)",
+                     "frac": achieved / hbm_peak,
+                     "traffic": GEMV_TRAFFIC_PER_LAUNCH_T16 if args.tokens == 16 else None,
+                     "kernel": "gemv_kernel (int4 decode)",
                      "us_per_launch": 1e6 * kern_s / (args.steps * n_calls),
                      "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": {"value": step_bytes * args.steps * world / e2e_elapsed / 1e9, "unit": "GB/s",
@@ -168,8 +177,8 @@ def cpu_baseline(tokens: int, budget_s: float = 12.0):
     except Exception:
         cores = 1
     done_bytes, t_total, n_calls, names = 0, 0.0, 0, []
-    for i, (name, n_in, n_out) in enumerate(PROJ):
-        seed = synth.layer_seed(2, i)
+    for i, (name, n_in, n_out) in enumerate(PROJ * 16):
+        seed = synth.layer_seed(2, i % len(PROJ))
         pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
         q, s, z = synth.w4_codes(n_out, n_in, seed)
         x = synth.activations(tokens, n_in, seed)
@@ -182,7 +191,7 @@ def cpu_baseline(tokens: int, budget_s: float = 12.0):
         if t_total > budget_s:
             break
     return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
-            "sample": f"{n_calls} projections ({'+'.join(names)}) of one layer, every output row, "
+            "sample": f"{n_calls} projection calls ({'+'.join(names)}) of one layer, every output row, "
                       f"{tokens} tokens, fp64 numpy ({t_total:.1f} s)"}
 
 

@@ -87,10 +87,10 @@ def test_rotate_parity(B, T, in_f, K, P):
 
 
 @pytest.mark.parametrize("in_f,K,P", [(4096, 8, 64), (14336, 16, 13), (384, 3, 64)])
-def test_rotate_decode_kernel_matches_general_kernel(B, in_f, K, P):
-    """Batches of at most 16 tokens take the decode rotation kernel (float4
-    exchange, packed f32x2 arithmetic); larger batches the general one. Both
-    apply the same operations in the same order: identical bits."""
+def test_rotate_kernels_agree_bit_for_bit(B, in_f, K, P):
+    """Batches of at most 16 tokens and of 256 or more take the quad kernel
+    (float4 exchange, packed f32x2 arithmetic); the others the general one.
+    All apply the same operations in the same order: identical bits."""
     seed = synth.layer_seed(1, 77 + K)
     pairs, theta, alpha = synth.rotation_params(in_f, K, seed, pairs_per_group=P)
     x = synth.activations(24, in_f, seed)
@@ -100,6 +100,12 @@ def test_rotate_decode_kernel_matches_general_kernel(B, in_f, K, P):
         small = host(B.paro_rotate(rot, dev(x[:T])))
         assert np.array_equal(small.view(np.uint16), big[:T].view(np.uint16)), T
     check_rotation(big[:16], x[:16], pairs, theta, alpha)
+    # batches of 256 tokens and more take the quad kernel with several quads per warp
+    x2 = synth.activations(300, in_f, seed + 1)
+    general = host(B.paro_rotate(rot, dev(x2[:255])))
+    quad = host(B.paro_rotate(rot, dev(x2)))
+    assert np.array_equal(quad[:255].view(np.uint16), general.view(np.uint16))
+    check_rotation(quad, x2, pairs, theta, alpha)
 
 
 @pytest.mark.parametrize("T", [2048, 8192])

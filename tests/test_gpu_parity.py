@@ -186,6 +186,8 @@ def _layer(B, in_f, out_f, K, P, seed, oracle_quant=True):
     (3, 384, 48, 8, 64),
     (8, 256, 80, 4, 13),
     (9, 384, 48, 1, 64),
+    (16, 128, 272, 2, 64),     # one group (half a 256-channel stage), ragged 128-row tile
+    (12, 640, 1040, 8, 64),    # odd stage count, many tiles split over CTAs
     (17, 512, 96, 8, 64),      # > 16 tokens: prefill path (tensor-core GEMM)
     (40, 384, 48, 8, 64),      # partial 128-row tile, odd group count
     (130, 512, 256, 8, 64),    # two 128-token tiles, ragged

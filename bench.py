@@ -34,7 +34,13 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "ParoQuant W4G128 linear: decode HBM GB/s, prefill TFLOP/s, % of roofline"
-PROJ = [("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672), ("down", 14336, 4096)]
+# decoder-layer linears (QKV and gate+up fused), by model shape
+MODELS = {
+    "llama3-8b": [("qkv", 4096, 6144), ("o", 4096, 4096), ("gate_up", 4096, 28672), ("down", 14336, 4096)],
+    "qwen3-4b": [("qkv", 2560, 6144), ("o", 4096, 2560), ("gate_up", 2560, 19456), ("down", 9728, 2560)],
+    "qwen3-14b": [("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 34816), ("down", 17408, 5120)],
+}
+PROJ = MODELS["llama3-8b"]
 K_LAYERS = 8
 GROUP = 128
 
@@ -142,7 +148,7 @@ def decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_byte
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16 (int4 weights, fp32 accumulate)",
-        "data": "synthetic (seeded Llama-3-8B-shaped layers; weights quantised on the GPU from T W)",
+        "data": f"synthetic (seeded {args.model}-shaped layers; weights quantised on the GPU from T W)",
         "config": config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
@@ -236,9 +242,9 @@ def run_reference(args, rank: int, world: int):
 
 
 def config(args):
-    return {"workload": f"llama3-8b decoder-layer W4G128 linears (qkv 4096x6144, o 4096x4096, "
-                        f"gate_up 4096x28672, down 14336x4096), decode {args.tokens} tokens, "
-                        f"K={K_LAYERS} rotation layers x 64 pairs/group",
+    shapes = ", ".join(f"{n} {i}x{o}" for n, i, o in PROJ)
+    return {"workload": f"{getattr(args, 'model', 'llama3-8b')} decoder-layer W4G128 linears ({shapes}), "
+                        f"decode {args.tokens} tokens, K={K_LAYERS} rotation layers x 64 pairs/group",
             "tokens": args.tokens, "layers_per_step": args.layers, "rotation_layers": K_LAYERS,
             "group": GROUP, "l2": f"inputs larger than L2: {args.layers} distinct layers per step",
             "parallelism": f"replicas x{args.gpus}"}
@@ -338,7 +344,7 @@ def bench_prefill(args, torch, B, local):
     except Exception:
         tc_peak = 1400.0
     tf = flops / times[False] / 1e12
-    print(json.dumps({"workload": f"prefill llama3-8b layer projections, {T} tokens, K={K_LAYERS}",
+    print(json.dumps({"workload": f"prefill {args.model} layer projections, {T} tokens, K={K_LAYERS}",
                       "ms_per_layer": 1e3 * times[True], "ms_per_layer_unrotated": 1e3 * times[False],
                       "TFLOP/s": flops / times[True] / 1e12, "TFLOP/s_gemm_only": tf,
                       "rotation_overhead": times[True] / times[False] - 1.0,
@@ -364,10 +370,14 @@ def main():
     ap.add_argument("--workload", default="decode", choices=["decode", "rotate", "prefill"],
                     help="decode: the headline step; rotate: paro_rotate alone (hidden 4096); "
                          "prefill: one layer's projections at --tokens (tensor-core GEMM)")
+    ap.add_argument("--model", default="llama3-8b", choices=sorted(MODELS),
+                    help="decoder-layer shapes (the headline line is llama3-8b)")
     ap.add_argument("--rot-k", type=int, default=8)
     ap.add_argument("--rot-pairs", type=int, default=64)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    global PROJ
+    PROJ = MODELS[args.model]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -32,7 +32,7 @@ def _rank_main(rank, world, port, outdir):
         # rank r is slower on one timer and faster on another
         mine = [1.0 + rank, 2.0 - rank, 0.5 + 0.25 * rank]
         got = bench.max_over_ranks(dist, mine)
-        args = types.SimpleNamespace(steps=10, warmup=3, tokens=16, layers=4, gpus=world)
+        args = types.SimpleNamespace(steps=10, warmup=3, tokens=16, layers=4, gpus=world, model="llama3-8b")
         line = bench.decode_line(args, world, got[0], got[1], got[2], step_bytes=1e9, gemv_bytes=5e8,
                                  n_calls=16, hbm_peak=6454.9, peak_kind="measured", h2d=1, d2h=2,
                                  per_proj={}, n_launch=320, clocks={})

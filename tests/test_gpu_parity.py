@@ -234,6 +234,45 @@ def test_linear_decode_full_size_sampled(B, T, in_f, out_f):
     check_linear(y[:, rows], x, pairs, theta, alpha, q[rows], s[rows], z[rows])
 
 
+# Qwen3-shaped decoder-layer linears: 4B-like (hidden 2560, intermediate 9728,
+# 32 q / 8 kv heads x 128) and 14B-like (hidden 5120, intermediate 17408,
+# 40 q / 8 kv heads x 128); QKV and gate+up fused.
+QWEN3 = [(2560, 6144), (4096, 2560), (2560, 19456), (9728, 2560),
+         (5120, 7168), (5120, 5120), (5120, 34816), (17408, 5120)]
+
+
+@pytest.mark.parametrize("T", [1, 8])
+@pytest.mark.parametrize("in_f,out_f", QWEN3)
+def test_linear_decode_qwen3_shapes_sampled(B, T, in_f, out_f):
+    seed = synth.layer_seed(4, in_f + out_f + T)
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+    q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
+    rows = np.random.default_rng(seed).choice(out_f, 128, replace=False)
+    rows[0], rows[-1] = 0, out_f - 1
+    check_linear(y[:, rows], x, pairs, theta, alpha, q[rows], s[rows], z[rows])
+
+
+@pytest.mark.parametrize("in_f,out_f", [(2560, 6144), (9728, 2560), (5120, 34816), (17408, 5120)])
+def test_linear_prefill_qwen3_shapes_sampled(B, in_f, out_f):
+    T = 4096
+    seed = synth.layer_seed(4, in_f + out_f)
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+    q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
+    rng = np.random.default_rng(seed)
+    toks = rng.choice(T, 16, replace=False)
+    toks[0], toks[-1] = 0, T - 1
+    rows = rng.choice(out_f, 128, replace=False)
+    check_linear(y[np.ix_(toks, rows)], x[toks], pairs, theta, alpha, q[rows], s[rows], z[rows])
+
+
 @pytest.mark.parametrize("in_f,out_f", [(4096, 4096), (14336, 4096)])
 def test_linear_prefill_full_size_sampled(B, in_f, out_f):
     T = 2048

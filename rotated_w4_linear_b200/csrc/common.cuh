@@ -46,8 +46,11 @@ __device__ __forceinline__ const uint8_t* rotx_block(const uint8_t* rotx, int t,
 // Quad exchange blocks for the decode rotation kernel, one per
 // (layer t, group g), 1280 B:
 //   [32 lanes][8 bytes]: float4-slot indices (0..127) in the warp's 2 KB
-//     exchange buffer where lane L stores channel 4L+j (bytes 0..3) and where
-//     it loads that channel's partner (bytes 4..7); a slot holds four tokens;
+//     exchange buffer where lane L stores channel 4L+j (bytes 0..3, bit 7
+//     set when the channel is in a pair of this layer) and where it loads
+//     that channel's partner (bytes 4..7); a slot holds four tokens. A
+//     channel in no pair (partial matchings) skips the exchange: its own
+//     value stands in for the partner, as in the rotation block (a = 1, b = 0);
 //   [32 lanes][float4]: (a, b) of channels 4L and 4L+1, as in the rotation block;
 //   [32 lanes][float4]: (a, b) of channels 4L+2 and 4L+3.
 // A 16-byte shared access is served a quarter-warp (8 lanes) at a time; the

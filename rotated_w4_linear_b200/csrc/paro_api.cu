@@ -239,8 +239,10 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
             uint8_t* x = &rotq[((size_t)t * G + g) * paro::kRotQBlockBytes];
             for (int l = 0; l < 32; ++l) {
                 for (int j = 0; j < 4; ++j) {
-                    x[8 * l + j] = (uint8_t)pos[4 * l + j];
-                    x[8 * l + 4 + j] = (uint8_t)pos[partner[4 * l + j]];
+                    const int c = 4 * l + j;
+                    // bit 7: the channel is in a pair of this layer (else it only keeps its value)
+                    x[8 * l + j] = (uint8_t)(pos[c] | (partner[c] != c ? 0x80 : 0));
+                    x[8 * l + 4 + j] = (uint8_t)pos[partner[c]];
                 }
             }
             for (int l = 0; l < 32; ++l) {   // (a, b) of channels 4l, 4l+1 | 4l+2, 4l+3

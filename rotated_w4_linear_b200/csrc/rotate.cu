@@ -212,10 +212,12 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
             const float4 c23 = *reinterpret_cast<const float4*>(blk + 768 + 16 * lane);
             const float ca[4] = {c01.x, c01.z, c23.x, c23.z}, cb[4] = {c01.y, c01.w, c23.y, c23.w};
             uint32_t st[4], ld[4];
+            bool act[4];                                   // channel in a pair of this layer
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                st[j] = 16u * ((pos.x >> (8 * j)) & 0xFFu);
-                ld[j] = 16u * ((pos.y >> (8 * j)) & 0xFFu);
+                st[j] = 16u * ((pos.x >> (8 * j)) & 0x7Fu);
+                ld[j] = 16u * ((pos.y >> (8 * j)) & 0x7Fu);
+                act[j] = (pos.x >> (8 * j + 7)) & 1u;
             }
 #pragma unroll
             for (int q = 0; q < QW; ++q) {
@@ -223,16 +225,23 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
                 // every lane has passed the barrier between (its reads precede it)
                 const uint32_t buf = xbuf + flip;
                 if (NBUF == 2) flip ^= 2048u;
+                // only channels in a pair go through shared memory (lanes
+                // with inactive channels drop out of those accesses)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(buf + st[j]), "l"(v[q][j][0]),
-                                 "l"(v[q][j][1]) : "memory");
+                    if (act[j])
+                        asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(buf + st[j]), "l"(v[q][j][0]),
+                                     "l"(v[q][j][1]) : "memory");
                 __syncwarp();
                 uint64_t p[4][2];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(p[j][0]), "=l"(p[j][1]) : "r"(buf + ld[j])
-                                 : "memory");
+                for (int j = 0; j < 4; ++j) {
+                    p[j][0] = v[q][j][0];
+                    p[j][1] = v[q][j][1];
+                    if (act[j])
+                        asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(p[j][0]), "=l"(p[j][1])
+                                     : "r"(buf + ld[j]) : "memory");
+                }
                 if (NBUF == 1) __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {

@@ -58,10 +58,10 @@ def call_bytes(T, n_in, n_out):
 
 
 # DRAM bytes (read + write) per decode-kernel launch, mean over the four
-# projections (qkv 13.24 MB, o 8.88 MB, gate+up 61.18 MB, down 30.99 MB), from
+# projections (qkv 13.24 MB, o 8.88 MB, gate+up 61.18 MB, down 31.00 MB), from
 # one ncu capture of the current kernel at 16 tokens; the command is in
 # profiles/gemv_kernel_gate_up_4096x28672_t16.md. None once the kernel changes.
-GEMV_TRAFFIC_PER_LAUNCH_T16 = (13238016 + 8875264 + 61180672 + 30993920) / 4
+GEMV_TRAFFIC_PER_LAUNCH_T16 = (13237248 + 8879104 + 61178368 + 30997504) / 4
 
 
 def peaks():

@@ -146,6 +146,16 @@ paro_status paro_linear(const paro_rot* rot, const void* X_dev,
                         void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,
                         void* workspace_dev, size_t workspace_bytes, paro_stream stream);
 
+/* paro_linear plus a bias: Y = (X T^-1) w_hat^T + b (CSDN article,
+ * section 2.1, Y = XW + b). bias_dev is fp16 [out_features] (2-byte
+ * aligned) or NULL; it is added to the fp32 sum before the single rounding
+ * to fp16. Arguments, workspace and errors as paro_linear. */
+paro_status paro_linear_bias(const paro_rot* rot, const void* X_dev,
+                             const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
+                             const void* bias_dev, void* Y_dev, int64_t tokens, int64_t in_features,
+                             int64_t out_features, void* workspace_dev, size_t workspace_bytes,
+                             paro_stream stream);
+
 /* paro_linear for decode batches (tokens <= 16) that allocates nothing and
  * takes no workspace: for callers that cannot allocate device memory, such
  * as a serving engine that hands all device memory to its own pool at start-

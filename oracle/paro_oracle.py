@@ -170,19 +170,24 @@ def quantize_layer(w: np.ndarray, pairs, theta, alpha, group: int = GROUP):
 # --------------------------------------------------------------------------
 # The layer
 # --------------------------------------------------------------------------
-def linear(x: np.ndarray, pairs, theta, alpha, q, s, z, group: int = GROUP) -> np.ndarray:
-    """Y = (X T^-1) w_hat^T in fp64, unrounded. x fp16/fp64 [T][in] -> [T][out]."""
+def linear(x: np.ndarray, pairs, theta, alpha, q, s, z, group: int = GROUP, bias=None) -> np.ndarray:
+    """Y = (X T^-1) w_hat^T (+ b) in fp64, unrounded. x fp16/fp64 [T][in] -> [T][out].
+    The bias b [out] is the "+ b" of CSDN article section 2.1 (Y = XW + b)."""
     xr = rotate_activations(x, pairs, theta, alpha, group)
-    return xr @ dequantize(q, s, z, group).astype(np.float64).T
+    y = xr @ dequantize(q, s, z, group).astype(np.float64).T
+    return y if bias is None else y + np.asarray(bias, dtype=np.float64)[None, :]
 
 
 def linear_fp16_pipeline(x: np.ndarray, pairs, theta, alpha, q, s, z, group: int = GROUP,
-                         round_output: bool = True) -> np.ndarray:
-    """The ideal fp16 pipeline: X' rounded to fp16, fp64 contraction with w_hat,
-    Y rounded to fp16 (or left in fp64 with round_output=False). Its distance
-    to `linear` is the format floor of any kernel that stores X' and Y in fp16."""
+                         round_output: bool = True, bias=None) -> np.ndarray:
+    """The ideal fp16 pipeline: X' rounded to fp16, fp64 contraction with w_hat
+    (+ b), Y rounded to fp16 (or left in fp64 with round_output=False). Its
+    distance to `linear` is the format floor of any kernel that stores X' and
+    Y in fp16."""
     xr = rotate_activations(x, pairs, theta, alpha, group).astype(np.float16).astype(np.float64)
     y = xr @ dequantize(q, s, z, group).astype(np.float64).T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
     return y.astype(np.float16) if round_output else y
 
 

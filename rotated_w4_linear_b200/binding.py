@@ -34,6 +34,7 @@ _SIGS = {
     "paro_quantize_weights": [_vp, _vp, _i64, _vp, _vp, _vp, _vp],
     "paro_linear_workspace_size": [_i64, _i64, _i64, ctypes.POINTER(_sz)],
     "paro_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
+    "paro_linear_bias": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
     "paro_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
     "paro_fault_status": [ctypes.POINTER(_int), _int],
     "paro_last_error": [],
@@ -195,6 +196,28 @@ def paro_linear(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_featur
     _check("paro_linear", lib().paro_linear(
         rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
         _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"),
+        _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
+        _stream(stream)))
+    return Y
+
+
+def paro_linear_bias(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, bias: Optional[torch.Tensor],
+                     out_features: int, Y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """paro_linear + bias (fp16 [out_features] CUDA tensor, or None)."""
+    T, in_f = X.shape
+    if Y is None:
+        Y = torch.empty((T, out_features), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(T, in_f, out_features, X.device)
+    b = None
+    if bias is not None:
+        if bias.numel() != out_features:
+            raise ValueError("bias must have out_features elements")
+        b = _dev(bias, torch.float16, "bias")
+    _check("paro_linear_bias", lib().paro_linear_bias(
+        rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
+        _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"), b,
         _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
         _stream(stream)))
     return Y

@@ -53,6 +53,7 @@ struct GemmArgs {
     int nsplit;                 // CTAs along z = cluster size along z (split-k)
     const uint32_t* sp;
     const uint8_t* zp;
+    const __half* bias;         // [out] fp16 or null
     __half* Y;
 };
 
@@ -210,10 +211,11 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 16; ++j) red[j * kRedStride + rloc] = __uint_as_float(r[j]);
                 } else if (row < a.out) {
+                    const float b = a.bias ? __half2float(a.bias[row]) : 0.f;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = n0 + c0 + j;
-                        if (t < a.T) a.Y[(size_t)t * a.out + row] = __float2half_rn(__uint_as_float(r[j]));
+                        if (t < a.T) a.Y[(size_t)t * a.out + row] = __float2half_rn(__uint_as_float(r[j]) + b);
                     }
                 }
             }
@@ -233,7 +235,8 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const int row = rb0 * 16 + rl;
             float sum = 0.f;
             for (int x = 0; x < a.nsplit; ++x) sum += ld_cluster_f32(red_addr + (uint32_t)(t * kRedStride + rl) * 4u, (uint32_t)x);
-            if (t < a.T && row < a.out) a.Y[(size_t)t * a.out + row] = __float2half_rn(sum);
+            if (t < a.T && row < a.out)
+                a.Y[(size_t)t * a.out + row] = __float2half_rn(sum + (a.bias ? __half2float(a.bias[row]) : 0.f));
         }
         cluster_barrier();                                // partial tiles stay alive until all reads are done
     } else {
@@ -323,7 +326,7 @@ bool encode_maps(const void* Xr, const void* qw, const void* sp, const void* zp,
                      (uint64_t)a.Gp * 8, 16u, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-GemmArgs make_args(int64_t T, int64_t in, int64_t out, const void* scp, const void* zp, void* Y) {
+GemmArgs make_args(int64_t T, int64_t in, int64_t out, const void* scp, const void* zp, const void* bias, void* Y) {
     GemmArgs a{};
     a.T = (int)T;
     a.in = (int)in;
@@ -336,17 +339,18 @@ GemmArgs make_args(int64_t T, int64_t in, int64_t out, const void* scp, const vo
     a.nsplit = 1;
     a.sp = static_cast<const uint32_t*>(scp);
     a.zp = static_cast<const uint8_t*>(zp);
+    a.bias = static_cast<const __half*>(bias);
     a.Y = static_cast<__half*>(Y);
     return a;
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, void* Y, int64_t T,
-                        int64_t in, int64_t out, cudaStream_t s) {
+cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, const void* bias, void* Y,
+                        int64_t T, int64_t in, int64_t out, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     const int BN = T <= 64 ? 64 : T <= 128 ? 128 : 256;
-    GemmArgs a = make_args(T, in, out, scp, zp, Y);
+    GemmArgs a = make_args(T, in, out, scp, zp, bias, Y);
     CUtensorMap tm[4];
     if (!encode_maps(Xr, qw, scp, zp, T, BN, a, tm)) return cudaErrorInvalidValue;
     const int mt = (a.nrb + 7) / 8;

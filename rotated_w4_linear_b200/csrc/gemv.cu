@@ -59,6 +59,7 @@ struct GemvArgs {
     const uint4* qw;
     const uint32_t* sp;
     const uint8_t* zp;
+    const __half* bias;   // [out] fp16 or null
     __half* Y;
 };
 
@@ -261,7 +262,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     if (a.nsplit == 1) {
         for (int i = threadIdx.x; i < a.T * nrows_tile; i += kWarps * 32) {
             const int t = i / nrows_tile, r = i - t * nrows_tile;
-            a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * SR + r]);
+            const float b = a.bias ? __half2float(a.bias[row0 + r]) : 0.f;
+            a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * SR + r] + b);
         }
         return;
     }
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
         const uint32_t off = red_local + (uint32_t)(t * SR + r) * 4u;
         float sum = 0.f;
         for (int x = 0; x < a.nsplit; ++x) sum += ld_dsmem(mapa(off, (uint32_t)x));
+        if (a.bias) sum += __half2float(a.bias[row0 + r]);
         a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(sum);
     }
     cluster_sync();                                        // tiles stay alive until every reader is done
@@ -424,7 +427,7 @@ cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStream_t s) 
 // null), then the decode kernel runs on it; both are programmatic dependent
 // launches, so the decode kernel's weight stream starts during the rotation.
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
-                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s) {
+                        const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -450,6 +453,7 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.qw = static_cast<const uint4*>(qw);
     a.sp = static_cast<const uint32_t*>(scp);
     a.zp = static_cast<const uint8_t*>(zp);
+    a.bias = static_cast<const __half*>(bias);
     a.Y = static_cast<__half*>(Y);
     cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, s) : launch_gemv_t<1>(a, p, s);
     if (e != cudaSuccess) return e;
@@ -500,7 +504,7 @@ cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw
     void* scratch = nullptr;
     cudaError_t e = noalloc_scratch(&scratch);
     if (e != cudaSuccess) return e;
-    return launch_gemv(rot, X, qw, scp, zp, Y, T, in, out, scratch, s);
+    return launch_gemv(rot, X, qw, scp, zp, nullptr, Y, T, in, out, scratch, s);
 }
 
 }  // namespace paro

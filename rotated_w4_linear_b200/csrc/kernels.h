@@ -35,7 +35,7 @@ cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t
 // Decode path (tokens <= 16): the decode rotation kernel into ws (when rot
 // is not null), then the int4 decode kernel, both programmatic dependent launches.
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
-                        void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s);
+                        const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s);
 
 // Decode with the X' scratch in a static device array (no allocation anywhere).
 size_t noalloc_scratch_bytes();
@@ -44,8 +44,8 @@ cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw
 
 // Prefill (tokens > 16): tcgen05 GEMM on X' (already rotated, in global memory),
 // launched as a programmatic dependent of the rotation kernel.
-cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, void* Y, int64_t T,
-                        int64_t in, int64_t out, cudaStream_t s);
+cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, const void* bias, void* Y,
+                        int64_t T, int64_t in, int64_t out, cudaStream_t s);
 
 // Fault code left by a bounded wait that ran out (0 = none); optionally cleared.
 cudaError_t read_fault(unsigned int* code, bool clear);

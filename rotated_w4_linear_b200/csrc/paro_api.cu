@@ -369,8 +369,9 @@ paro_status paro_linear_workspace_size(int64_t T, int64_t in, int64_t out, size_
     return PARO_OK;
 }
 
-paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp, void* Y,
-                        int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes, paro_stream stream) {
+paro_status paro_linear_bias(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
+                             const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws,
+                             size_t ws_bytes, paro_stream stream) {
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
@@ -380,6 +381,7 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
     if (!X || !qw || !sp || !zp || !Y || !ws) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(X) || !aligned16(qw) || !aligned16(sp) || !aligned16(zp) || !aligned16(Y) || !aligned16(ws))
         return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return fail(PARO_ERR_ARG, "bias must be 2-byte aligned");
     if (T > (1LL << 31) / in) return fail(PARO_ERR_UNSUPPORTED, "tokens too large");
     size_t need = 0;
     paro_linear_workspace_size(T, in, out, &need);
@@ -388,7 +390,7 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
     const paro::RotDev* rd = r ? &r->dev : nullptr;
     cudaError_t e;
     if (T <= 16) {   // decode rotation kernel into ws, then the int4 decode kernel
-        e = paro::launch_gemv(rd, X, qw, sp, zp, Y, T, in, out, ws, s);
+        e = paro::launch_gemv(rd, X, qw, sp, zp, bias, Y, T, in, out, ws, s);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
     // X' = X T^-1 into the workspace, then the tensor-core GEMM as a
@@ -399,8 +401,13 @@ paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const 
         if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
         src = ws;
     }
-    e = paro::launch_gemm(src, qw, sp, zp, Y, T, in, out, s);
+    e = paro::launch_gemm(src, qw, sp, zp, bias, Y, T, in, out, s);
     return e == cudaSuccess ? PARO_OK : cuda_fail(e, "prefill launch");
+}
+
+paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp, void* Y,
+                        int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes, paro_stream stream) {
+    return paro_linear_bias(r, X, qw, sp, zp, nullptr, Y, T, in, out, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

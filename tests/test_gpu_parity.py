@@ -48,13 +48,13 @@ def check_rotation(got16, x, pairs, theta, alpha):
     return fl
 
 
-def check_linear(y16, x, pairs, theta, alpha, q, s, z):
+def check_linear(y16, x, pairs, theta, alpha, q, s, z, bias=None):
     if pairs is None:                       # unrotated layer: theta = 0, alpha = 1
         pairs, theta, alpha = synth.rotation_params(x.shape[1], 1, 0)
         theta = np.zeros_like(theta)
         alpha = np.ones_like(alpha)
-    ref = O.linear(x, pairs, theta, alpha, q, s, z)
-    x16 = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, round_output=False)
+    ref = O.linear(x, pairs, theta, alpha, q, s, z, bias=bias)
+    x16 = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, round_output=False, bias=bias)
     y = y16.astype(np.float64)
     rel, mx = O.output_errors(y, ref)
     ulp = np.abs(np.spacing(np.abs(ref).astype(np.float16))).astype(np.float64)
@@ -205,6 +205,20 @@ def test_linear_parity_exhaustive(B, T, in_f, out_f, K, P):
         y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f, ws=ws))
         check_linear(y, x, pairs, theta, alpha, q, s, z)
     assert B.paro_fault_status() == 0
+
+
+@pytest.mark.parametrize("T,in_f,out_f", [(1, 512, 96), (16, 384, 272), (40, 512, 160), (300, 256, 48)])
+def test_linear_bias(B, T, in_f, out_f):
+    """Y = (X T^-1) w_hat^T + b on the decode (T <= 16) and prefill paths."""
+    seed = synth.layer_seed(5, T + in_f)
+    (pairs, theta, alpha, q, s, z), (qw, sp, zp) = _layer(B, in_f, out_f, 8, 64, seed)
+    x = synth.activations(T, in_f, seed)
+    b = (np.random.default_rng(seed).standard_normal(out_f) * 4).astype(np.float16)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = host(B.paro_linear_bias(rot, dev(x), qw, sp, zp, dev(b), out_f))
+    check_linear(y, x, pairs, theta, alpha, q, s, z, bias=b)
+    y0 = host(B.paro_linear_bias(rot, dev(x), qw, sp, zp, None, out_f))       # null bias = paro_linear
+    assert np.array_equal(y0.view(np.uint16), host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f)).view(np.uint16))
 
 
 @pytest.mark.parametrize("T", [1, 5, 16])

@@ -249,3 +249,24 @@ def test_error_measures():
     assert np.isclose(fl, 1e-5 / 0.02) and np.isclose(lit, 1e-2)
     rel, mx = O.output_errors(np.array([3.0, 4.0]), np.array([3.0, 4.5]))
     assert np.isclose(mx, 0.5) and np.isclose(rel, 0.5 / np.hypot(3, 4.5))
+
+
+def test_bias_is_added_once_per_output_column():
+    """CSDN article, section 2.1: Y = XW + b. With zero codes at zero point
+    0 and any scale (w_hat = 0) the layer returns exactly b on every row;
+    for real codes, adding b shifts each column by b and nothing else."""
+    rng = np.random.default_rng(7)
+    T, in_f, out_f = 3, 256, 40
+    pairs, theta, alpha = synth.rotation_params(in_f, 2, 11)
+    x = synth.activations(T, in_f, 11)
+    b = rng.standard_normal(out_f).astype(np.float16)
+    q0 = np.zeros((out_f, in_f), np.uint8)
+    z0 = np.zeros((out_f, in_f // 128), np.uint8)
+    s0 = np.full((out_f, in_f // 128), 0.5, np.float16)
+    y0 = O.linear(x, pairs, theta, alpha, q0, s0, z0, bias=b)
+    assert np.array_equal(y0, np.broadcast_to(b.astype(np.float64), (T, out_f)))
+    q, s, z = synth.w4_codes(out_f, in_f, 12)
+    ya = O.linear(x, pairs, theta, alpha, q, s, z)
+    yb = O.linear(x, pairs, theta, alpha, q, s, z, bias=b)
+    bb = np.broadcast_to(b.astype(np.float64), (T, out_f))
+    assert np.all(np.abs((yb - ya) - bb) <= 1e-12 * (np.abs(ya) + np.abs(bb)))

@@ -259,24 +259,30 @@ def bench_rotate(args, torch, B, local):
     T, n_in, K, P = args.tokens, 4096, args.rot_k, args.rot_pairs
     pairs, theta, alpha = synth.rotation_params(n_in, K, synth.layer_seed(1, K), pairs_per_group=P)
     rot = B.paro_rot_create(pairs, theta, alpha)
-    copies = max(1, (512 << 20) // (4 * T * n_in))
+    copies = min(64, max(1, (512 << 20) // (4 * T * n_in)))   # > L2 for T >= 256
     xs = [torch.from_numpy(synth.activations(T, n_in, synth.layer_seed(1, c))).cuda() for c in range(copies)]
     ys = [torch.empty_like(x) for x in xs]
     stream = torch.cuda.current_stream()
+    # one pass over the copies captured in a CUDA graph: small batches are
+    # timed without the host's per-call launch cost
+    for x, y in zip(xs, ys):
+        B.paro_rotate(rot, x, y)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for x, y in zip(xs, ys):
+            B.paro_rotate(rot, x, y)
     for _ in range(args.warmup):
-        for x, y in zip(xs, ys):
-            B.paro_rotate(rot, x, y)
+        g.replay()
     torch.cuda.synchronize()
-    evs = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
     for _ in range(args.steps):
-        for x, y in zip(xs, ys):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            B.paro_rotate(rot, x, y)
-            e1.record(stream)
-            evs.append((e0, e1))
+        g.replay()
+    e1.record(stream)
     torch.cuda.synchronize()
-    per = sum(a.elapsed_time(b) for a, b in evs) / 1e3 / len(evs)
+    per = e0.elapsed_time(e1) / 1e3 / (args.steps * len(xs))
+    del g
     nbytes = 4 * T * n_in + K * (n_in // GROUP) * P * 10 + 4 * n_in
     hbm_peak, _, kind = peaks()
     print(json.dumps({"workload": f"paro_rotate tokens={T} hidden={n_in} K={K} pairs/group={P}",

@@ -45,6 +45,7 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kStages = 3;
+constexpr int kMaxSplit = 16;                             // largest cluster (k-chunks per row tile)
 constexpr int kItemGroups = 2;                            // groups per item
 constexpr int kItemQBytes = kItemGroups * 2 * 512;        // int4 codes
 constexpr int kItemBytes = kItemQBytes + kItemGroups * 32 + 16;   // + scales + zeros
@@ -90,9 +91,10 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 ld_dsmem4(uint32_t addr) {   // 16-byte aligned
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr) : "memory");
     return v;
 }
 __device__ __forceinline__ void cluster_sync() {
@@ -163,16 +165,21 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     // ---- X' chunk and partial tile (waits for the previous grid: X' may be its output)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
+        // all of the chunk's 16-byte copies are in flight at once (cp.async;
+        // rows >= T are zero-filled by a source size of 0), then one wait
         const int vec_per_row = ncg * 16;
         const int total = NT * 8 * vec_per_row;
+        const __half* xsrc = a.Xr + (size_t)g_begin * 128;
         for (int i = threadIdx.x; i < total; i += kWarps * 32) {
             const int tok = i / vec_per_row, v = i - tok * vec_per_row;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (tok < a.T)
-                val = __ldg(reinterpret_cast<const uint4*>(a.Xr + (size_t)tok * a.in + (size_t)g_begin * 128) + v);
-            *reinterpret_cast<uint4*>(xs + (size_t)tok * XS + v * 8) = val;
+            const bool real = tok < a.T;
+            const void* src = reinterpret_cast<const uint4*>(xsrc + (size_t)(real ? tok : 0) * a.in) + v;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(xs + (size_t)tok * XS + v * 8)),
+                         "l"(src), "r"(real ? 16 : 0) : "memory");
         }
+        cp_async_commit();
         for (int i = threadIdx.x; i < NT * 8 * SR; i += kWarps * 32) red[i] = 0.f;
+        cp_async_wait<0>();                                // (the first weight items are in by now too)
     }
     __syncthreads();
 
@@ -271,13 +278,33 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) 
     const int rlo = chunk * a.share;
     const int n = max(0, min(a.share, nrows_tile - rlo));
     const uint32_t red_local = smem_u32(red);
-    for (int i = threadIdx.x; i < a.T * n; i += kWarps * 32) {
-        const int t = i / n, r = rlo + (i - t * n);
+    // four rows per thread (n is a multiple of 16); the loads from all the
+    // cluster's tiles are issued before any is used, so their latencies overlap
+    const int n4 = n >> 2;
+    for (int i = threadIdx.x; i < a.T * n4; i += kWarps * 32) {
+        const int t = i / n4, r = rlo + 4 * (i - t * n4);
         const uint32_t off = red_local + (uint32_t)(t * SR + r) * 4u;
-        float sum = 0.f;
-        for (int x = 0; x < a.nsplit; ++x) sum += ld_dsmem(mapa(off, (uint32_t)x));
-        if (a.bias) sum += __half2float(a.bias[row0 + r]);
-        a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(sum);
+        float4 part[kMaxSplit];
+#pragma unroll
+        for (int x = 0; x < kMaxSplit; ++x)
+            if (x < a.nsplit) part[x] = ld_dsmem4(mapa(off, (uint32_t)x));
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int x = 0; x < kMaxSplit; ++x)
+            if (x < a.nsplit) {
+                sum.x += part[x].x;
+                sum.y += part[x].y;
+                sum.z += part[x].z;
+                sum.w += part[x].w;
+            }
+        if (a.bias) {
+            sum.x += __half2float(a.bias[row0 + r]);
+            sum.y += __half2float(a.bias[row0 + r + 1]);
+            sum.z += __half2float(a.bias[row0 + r + 2]);
+            sum.w += __half2float(a.bias[row0 + r + 3]);
+        }
+        *reinterpret_cast<uint2*>(a.Y + (size_t)t * a.out + row0 + r) =
+            make_uint2(pack_half2(sum.x, sum.y), pack_half2(sum.z, sum.w));
     }
     cluster_sync();                                        // tiles stay alive until every reader is done
 }

@@ -2,7 +2,7 @@
 // already in global memory (written by the rotation kernel launched just
 // before on the same stream). The int4 weight stream dominates: HBM bound.
 //
-// Launch: a grid of (nsplit, rowtiles) CTAs of 8 warps; CTAs with the same
+// Launch: a grid of (nsplit, rowtiles) CTAs of 16 warps, one per SM; CTAs with the same
 // row tile form one thread-block cluster along x, each owning a k-chunk of
 // KC 128-channel groups. The kernel is a programmatic dependent launch: it
 // starts while the kernel before it still runs, streams its first weights,
@@ -11,7 +11,7 @@
 //
 //   work split: the CTA's items (one row block of 16 rows x two groups: 2 KB
 //     of int4 codes + scales + zeros) in row-block-major order are cut into
-//     eight equal contiguous runs, one per warp;
+//     sixteen equal contiguous runs, one per warp;
 //   weight stream: each warp streams its run through a private 3-stage
 //     shared-memory ring with cp.async (16-byte global->shared copies that
 //     bypass the registers): one commit group per item, wait on the oldest,
@@ -43,7 +43,7 @@ namespace paro {
 
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr int kStages = 3;
 constexpr int kMaxSplit = 16;                             // largest cluster (k-chunks per row tile)
 constexpr int kItemGroups = 2;                            // groups per item
@@ -119,7 +119,7 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, uint32_t slot, int
 }  // namespace
 
 template <int NT>
-__global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) {
     // the next kernel on the stream may launch now: it prefetches only its
     // weights before it waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;");
@@ -380,9 +380,11 @@ GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
         for (int RT = 1; RT <= std::min(nrb, 64); ++RT) {
             const size_t smem = gemv_smem(NT, KC, RT);
             if (smem > 200 * 1024) break;
-            // two CTAs per SM, with room beside them for one CTA of the
-            // rotation kernel that runs before this one
-            const int per_sm = (2 * (smem + kReserved) + rot_reserve <= kSmemPerSm) ? 2 : 1;
+            // one CTA of 16 warps per SM (one copy of the X' chunk per SM),
+            // with room beside it for one CTA of the rotation kernel that
+            // runs before this one
+            if (smem + kReserved + rot_reserve > kSmemPerSm) break;
+            const int per_sm = 1;
             const int slots = gemv_slots<NT>(dev, ns, per_sm);
             const int rowtiles = (nrb + RT - 1) / RT;
             const int ctas = ns * rowtiles;

@@ -365,7 +365,7 @@ template <int NT>
 GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
     const int G = (int)(in / 128);
     const int nrb = (int)(out / 16);
-    const int kc_max = NT == 2 ? 10 : 20;                 // X' chunk <= ~41 KB
+    const int kc_max = NT == 2 ? 20 : 40;                 // X' chunk <= ~82 KB (one CTA per SM)
     constexpr size_t kSmemPerSm = 228 * 1024, kReserved = 1024;
     const size_t rot_reserve = K > 0 ? rotate_decode_smem(K, T) + kReserved : 0;
     GemvPlan best{};

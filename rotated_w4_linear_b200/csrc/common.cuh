@@ -9,8 +9,9 @@
 namespace paro {
 
 // ---------------------------------------------------------------------------
-// Prepared rotation parameters ("rotation block"), one per (layer t, group g),
-// 1152 bytes: 128 partner bytes, then 128 float2 (a, b).
+// Prepared rotation parameters ("rotation block", host image from which the
+// device exchange blocks below are built), one per (layer t, group g), 1152
+// bytes: 128 partner bytes, then 128 float2 (a, b).
 // Channel c of the group becomes a * v[c] + b * v[partner[c]]:
 //   first channel i of a pair (i, j, th): a = cos th, b = -sin th, partner j
 //   second channel j:                     a = cos th, b = +sin th, partner i
@@ -19,10 +20,6 @@ namespace paro {
 // written per output channel.
 // ---------------------------------------------------------------------------
 constexpr int kRotBlockBytes = 128 + 128 * 8;
-
-__device__ __forceinline__ const uint8_t* rot_block(const uint8_t* rotp, int t, int g, int G) {
-    return rotp + ((size_t)t * G + g) * kRotBlockBytes;
-}
 
 // ---------------------------------------------------------------------------
 // Exchange blocks for the rotation kernel, one per (layer t, group g), 1536 B:
@@ -99,12 +96,6 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 // Zeros:  uint8  [out/16][Gp][8] with Gp = G rounded up to even (two groups'
 //         zeros form one aligned 16-byte copy), byte g = (z[row g] | z[row g+8] << 4).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t nib_pair_to_f16x2(uint32_t w) {
-    // (w & 0x000f000f) | 0x64006400: fp16 bit patterns of 1024 + nibble
-    uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x000f000fu), "r"(0x64006400u));
-    return r;
-}
 
 __device__ __forceinline__ uint32_t hsub2_rn(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -146,11 +137,6 @@ __device__ __forceinline__ Zero2 zero_consts(uint32_t zbyte) {
     return r;
 }
 
-// zero byte (z0 | z1 << 4) -> fp16x2 (1024 + z, 1024 + z) for z0 (lo) and z1 (hi)
-__device__ __forceinline__ void zero_bias(uint32_t zbyte, uint32_t& zb0, uint32_t& zb1) {
-    zb0 = ((zbyte & 0xFu) | 0x6400u) * 0x00010001u;
-    zb1 = (((zbyte >> 4) & 0xFu) | 0x6400u) * 0x00010001u;
-}
 
 // scale word (s0 | s1 << 16) -> (s0, s0) and (s1, s1)
 __device__ __forceinline__ void scale_pairs(uint32_t sw, uint32_t& sc0, uint32_t& sc1) {
@@ -176,11 +162,6 @@ __device__ __forceinline__ void dequant_word(uint32_t w, const Zero2& z, uint32_
     h[3] = hmul2_rn(hfma2_rn(lop3_and_or(w8, 0x00F000F0u, kMagic), kSixteenth, z.zc1), sc1);
 }
 
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-    return v;
-}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -197,40 +178,10 @@ __device__ __forceinline__ uint32_t lds8(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-    return r;
-}
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// ---------------------------------------------------------------------------
-// One warp rotates one 128-channel group of one token held as 4 channels per
-// lane (lane L: channels 4L..4L+3). `buf` is 128 floats of warp-private shared
-// memory. Applies layers t = 0..K-1 of group g.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void rotate_group_warp(float v[4], const uint8_t* rotp, int g, int G, int K,
-                                                  float* buf, int lane) {
-    for (int t = 0; t < K; ++t) {
-        const uint8_t* blk = rot_block(rotp, t, g, G);
-        const uint32_t pw = __ldg(reinterpret_cast<const uint32_t*>(blk) + lane);
-        const float4 c01 = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane);
-        const float4 c23 = __ldg(reinterpret_cast<const float4*>(blk + 128) + 2 * lane + 1);
-        *reinterpret_cast<float4*>(buf + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
-        __syncwarp();
-        const float p0 = buf[pw & 0xFF], p1 = buf[(pw >> 8) & 0xFF];
-        const float p2 = buf[(pw >> 16) & 0xFF], p3 = buf[pw >> 24];
-        __syncwarp();
-        v[0] = fmaf(c01.y, p0, c01.x * v[0]);
-        v[1] = fmaf(c01.w, p1, c01.z * v[1]);
-        v[2] = fmaf(c23.y, p2, c23.x * v[2]);
-        v[3] = fmaf(c23.w, p3, c23.z * v[3]);
-    }
 }
 
 }  // namespace paro

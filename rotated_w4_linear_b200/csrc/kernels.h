@@ -11,7 +11,6 @@ struct RotDev {
     int G = 0;              // groups of 128
     int K = 0;              // rotation layers
     int P = 0;              // active pairs per (layer, group)
-    uint8_t* rotp = nullptr;       // [K][G] rotation blocks (fp32 coefficients)
     uint8_t* rotx = nullptr;       // [K][G] exchange blocks: conflict-free positions + coefficients
     uint8_t* rotq = nullptr;       // [K][G] quad exchange blocks (decode prologue)
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha

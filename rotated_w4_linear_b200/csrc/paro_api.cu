@@ -258,8 +258,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
         alpha64[c] = (double)alpha[c];
     }
 
-    const size_t o_rot32 = 0;
-    const size_t o_inv = o_rot32 + round256(rot32.size());
+    const size_t o_inv = 0;
     const size_t o_rot64 = o_inv + round256(inv_alpha.size() * sizeof(float));
     const size_t o_a64 = o_rot64 + round256(rot64.size());
     const size_t o_rotx = o_a64 + round256(alpha64.size() * sizeof(double));
@@ -272,8 +271,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     cudaError_t e = cudaMalloc(&r->block, total);
     if (e != cudaSuccess) { delete r; return cuda_fail(e, "cudaMalloc(rotation tables)"); }
     char* base = static_cast<char*>(r->block);
-    e = cudaMemcpy(base + o_rot32, rot32.data(), rot32.size(), cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemcpy(base + o_inv, inv_alpha.data(), inv_alpha.size() * 4, cudaMemcpyHostToDevice);
+    e = cudaMemcpy(base + o_inv, inv_alpha.data(), inv_alpha.size() * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_rot64, rot64.data(), rot64.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !rotx.empty()) e = cudaMemcpy(base + o_rotx, rotx.data(), rotx.size(), cudaMemcpyHostToDevice);
@@ -283,7 +281,6 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     r->dev.G = G;
     r->dev.K = K;
     r->dev.P = P;
-    r->dev.rotp = reinterpret_cast<uint8_t*>(base + o_rot32);
     r->dev.inv_alpha = reinterpret_cast<float*>(base + o_inv);
     r->dev.rotp64 = reinterpret_cast<uint8_t*>(base + o_rot64);
     r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);

@@ -101,18 +101,35 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Copy one item (row block rb, groups g0, g0+1 if ng == 2) into a ring slot.
-__device__ __forceinline__ void issue_item(const GemvArgs& a, uint32_t slot, int rb, int g0, int ng, int lane) {
+// A lane's source pointers for the items of one row block: codes (the
+// lane's 16 bytes of each 512-byte k block), scales (lanes 0..3: 16 bytes
+// each) and zeros (lane 31: the item's 16 bytes). Within a row block the
+// next item is 2 KB, 64 B and 16 B further on.
+struct ItemSrc {
+    const uint4* q;
+    const uint32_t* sc;
+    const uint8_t* z;
+};
+
+__device__ __forceinline__ ItemSrc item_src(const GemvArgs& a, int rb, int g0, int lane) {
     const int nkb = a.in >> 6;
-    const uint4* q = a.qw + ((size_t)rb * nkb + 2 * g0) * 32;
+    ItemSrc p;
+    p.q = a.qw + ((size_t)rb * nkb + 2 * g0) * 32 + lane;
+    p.sc = a.sp + ((size_t)rb * a.G + g0) * 8 + lane * 4;
+    p.z = a.zp + ((size_t)rb * a.Gp + g0) * 8;
+    return p;
+}
+
+// Copy one item (groups g0, g0+1 if ng == 2 of the source's row block) into
+// a ring slot; `dst` is the slot address plus this lane's 16-byte offset.
+__device__ __forceinline__ void issue_item(const ItemSrc& p, uint32_t slot, uint32_t dst, int ng, int lane) {
 #pragma unroll
     for (int kb = 0; kb < 2 * kItemGroups; ++kb)
-        if (kb < 2 * ng) cp_async16(slot + kb * 512 + lane * 16, q + kb * 32 + lane);
-    if (lane < 2 * ng) cp_async16(slot + kItemQBytes + lane * 16, a.sp + ((size_t)rb * a.G + g0) * 8 + lane * 4);
+        if (kb < 2 * ng) cp_async16(dst + kb * 512, p.q + kb * 32);
+    if (lane < 2 * ng) cp_async16(slot + kItemQBytes + lane * 16, p.sc);
     if (lane == 31) {
-        const uint8_t* z = a.zp + ((size_t)rb * a.Gp + g0) * 8;
-        if (ng == 2) cp_async16(slot + kItemQBytes + kItemGroups * 32, z);
-        else cp_async8(slot + kItemQBytes + kItemGroups * 32, z);
+        if (ng == 2) cp_async16(slot + kItemQBytes + kItemGroups * 32, p.z);
+        else cp_async8(slot + kItemQBytes + kItemGroups * 32, p.z);
     }
 }
 
@@ -139,19 +156,30 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     const int i_lo = (int)(((int64_t)items * warp) / kWarps);
     const int nmine = (int)(((int64_t)items * (warp + 1)) / kWarps) - i_lo;
 
-    const int XS = a.KC * 128 + 16;                        // halves; row stride == 8 words mod 32
+    const int XS = a.KC * 128 + 8;                         // halves; row stride == 16 bytes mod 128
     const int SR = a.RT * 16 + 4;                          // floats per token row of the partial tile
     __half* xs = reinterpret_cast<__half*>(smem);
     float* red = reinterpret_cast<float*>(smem + (size_t)NT * 8 * XS * 2);
     unsigned char* ring = reinterpret_cast<unsigned char*>(red + NT * 8 * SR);
     const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kStages * kItemBytes);
 
-    // producer cursor: (row block, sub) of the next item to copy
+    // producer cursor: (row block, sub) of the next item to copy and the
+    // lane's source pointers, advanced incrementally
     int p_rb = rb_begin + (nsub ? i_lo / nsub : 0), p_sub = nsub ? i_lo % nsub : 0;
+    ItemSrc src = item_src(a, p_rb, g_begin + p_sub * kItemGroups, lane);
     auto issue_next = [&](int stage) {
         const int g0 = g_begin + p_sub * kItemGroups;
-        issue_item(a, ring_w + stage * kItemBytes, p_rb, g0, min(kItemGroups, g_end - g0), lane);
-        if (++p_sub == nsub) { p_sub = 0; ++p_rb; }
+        const uint32_t slot = ring_w + stage * kItemBytes;
+        issue_item(src, slot, slot + lane * 16, min(kItemGroups, g_end - g0), lane);
+        if (++p_sub == nsub) {
+            p_sub = 0;
+            ++p_rb;
+            src = item_src(a, p_rb, g_begin, lane);
+        } else {
+            src.q += kItemGroups * 2 * 32;
+            src.sc += kItemGroups * 8;
+            src.z += kItemGroups * 8;
+        }
     };
 
     // ---- weight stream prologue: first kStages-1 items in flight (weights
@@ -165,17 +193,22 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     // ---- X' chunk and partial tile (waits for the previous grid: X' may be its output)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
-        // all of the chunk's 16-byte copies are in flight at once (cp.async;
-        // rows >= T are zero-filled by a source size of 0), then one wait
-        const int vec_per_row = ncg * 16;
-        const int total = NT * 8 * vec_per_row;
+        // all of the chunk's copies are in flight at once (cp.async; rows
+        // >= T are zero-filled by a source size of 0), then one wait. Within
+        // each 64-channel block the row is stored lane-major: channel
+        // 16 j + 4 q + e at position 16 q + 4 j + e, so lane q of a fragment
+        // row finds the four k tiles' B values in 32 contiguous bytes.
+        const int pieces_per_row = ncg * 32;                // 8-byte pieces of 4 channels
+        const int total = NT * 8 * pieces_per_row;
         const __half* xsrc = a.Xr + (size_t)g_begin * 128;
         for (int i = threadIdx.x; i < total; i += kWarps * 32) {
-            const int tok = i / vec_per_row, v = i - tok * vec_per_row;
+            const int tok = i / pieces_per_row, v = i - tok * pieces_per_row;   // v: 4-channel piece
+            const int blk = v >> 4, jq = v & 15, j = jq >> 2, q = jq & 3;       // channel 64 blk + 16 j + 4 q
             const bool real = tok < a.T;
-            const void* src = reinterpret_cast<const uint4*>(xsrc + (size_t)(real ? tok : 0) * a.in) + v;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(xs + (size_t)tok * XS + v * 8)),
-                         "l"(src), "r"(real ? 16 : 0) : "memory");
+            const __half* src = xsrc + (size_t)(real ? tok : 0) * a.in + 4 * v;
+            const uint32_t dst = smem_u32(xs + (size_t)tok * XS + blk * 64 + 16 * q + 4 * j);
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(real ? 8 : 0)
+                         : "memory");
         }
         cp_async_commit();
         for (int i = threadIdx.x; i < NT * 8 * SR; i += kWarps * 32) red[i] = 0.f;
@@ -192,7 +225,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     const unsigned char* xrow[NT];                         // this lane's B rows
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
-        xrow[nt] = reinterpret_cast<const unsigned char*>(xs + (size_t)(nt * 8 + gq) * XS + 4 * qd);
+        xrow[nt] = reinterpret_cast<const unsigned char*>(xs + (size_t)(nt * 8 + gq) * XS + 16 * qd);
     const unsigned char* ring_p = ring + (size_t)warp * kStages * kItemBytes;
     float acc[NT][2][4];
 #pragma unroll
@@ -235,16 +268,23 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
                 for (int h = 0; h < 2; ++h) {
                     const uint4 wv = *reinterpret_cast<const uint4*>(slot + (2 * g + h) * 512 + lane * 16);
                     const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                    // B values of the block's four k tiles: two 16-byte loads per token tile
+                    const int bbyte = kb_off + (g * 128 + h * 64) * 2;
+                    uint4 bq[NT][2];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        bq[nt][0] = *reinterpret_cast<const uint4*>(xrow[nt] + bbyte);
+                        bq[nt][1] = *reinterpret_cast<const uint4*>(xrow[nt] + bbyte + 16);
+                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         uint32_t hh[4];
                         dequant_word(words[j], zc, sc0, sc1, hh);
                         const uint32_t A[4] = {hh[0], hh[2], hh[1], hh[3]};
-                        const int kbyte = kb_off + (g * 128 + h * 64 + j * 16) * 2;
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            const uint2 bv = *reinterpret_cast<const uint2*>(xrow[nt] + kbyte);
-                            mma16816(acc[nt][j & 1], A, bv.x, bv.y);
+                            const uint4& b4 = bq[nt][j >> 1];
+                            mma16816(acc[nt][j & 1], A, (j & 1) ? b4.z : b4.x, (j & 1) ? b4.w : b4.y);
                         }
                     }
                 }
@@ -317,7 +357,7 @@ struct GemvPlan {
 };
 
 size_t gemv_smem(int NT, int KC, int RT) {
-    return (size_t)NT * 8 * (KC * 128 + 16) * 2 + (size_t)NT * 8 * (RT * 16 + 4) * 4 +
+    return (size_t)NT * 8 * (KC * 128 + 8) * 2 + (size_t)NT * 8 * (RT * 16 + 4) * 4 +
            (size_t)kWarps * kStages * kItemBytes;
 }
 

@@ -137,9 +137,14 @@ __device__ __forceinline__ void issue_item(const ItemSrc& p, uint32_t slot, uint
 
 template <int NT>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) {
-    // the next kernel on the stream may launch now: it prefetches only its
-    // weights before it waits for this grid to complete
-    asm volatile("griddepcontrol.launch_dependents;");
+    // When the next kernel on the stream may launch (it prefetches only its
+    // weights, or its tables, before it waits for this grid to complete):
+    // at 8 tokens or fewer right away; above that after the mainloop, so that
+    // the next rotation kernel's CTAs land on SMs as this grid's CTAs leave
+    // instead of crowding the few SMs this grid left free (measured: the
+    // early trigger costs 1.5-2 us per projection at 16 tokens, the late one
+    // 0.5-1 us at 1 token).
+    if (NT == 1) asm volatile("griddepcontrol.launch_dependents;");
     extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int chunk = blockIdx.x, rt = blockIdx.y;
@@ -299,6 +304,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         }
     }
     if (nmine > 0 && c_sub != 0) flush(c_rbl);             // run ended inside a row block
+    if (NT == 2) asm volatile("griddepcontrol.launch_dependents;");
     cp_async_wait<0>();
     __syncthreads();
 

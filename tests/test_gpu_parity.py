@@ -249,6 +249,28 @@ def test_linear_decode_full_size_sampled(B, T, in_f, out_f):
     check_linear(y[:, rows], x, pairs, theta, alpha, q[rows], s[rows], z[rows])
 
 
+def _random_shapes(n, seed):
+    rng = np.random.default_rng(seed)
+    for _ in range(n):
+        yield (int(rng.integers(1, 17)), 128 * int(rng.integers(1, 97)), 16 * int(rng.integers(1, 769)))
+
+
+@pytest.mark.parametrize("T,in_f,out_f", list(_random_shapes(12, 2024)))
+def test_linear_decode_random_shapes_sampled(B, T, in_f, out_f):
+    """The decode planner's tilings (k-chunk, cluster size, row tile, token
+    tiles) on random shapes up to 12288 inputs and 12288 outputs."""
+    seed = synth.layer_seed(6, T + in_f + out_f)
+    pairs, theta, alpha = synth.rotation_params(in_f, 4, seed, pairs_per_group=48)
+    q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
+    rows = np.unique(np.concatenate([[0, out_f - 1], np.random.default_rng(seed).choice(out_f, min(out_f, 96), replace=False)]))
+    check_linear(y[:, rows], x, pairs, theta, alpha, q[rows], s[rows], z[rows])
+    assert B.paro_fault_status() == 0
+
+
 # Qwen3-shaped decoder-layer linears: 4B-like (hidden 2560, intermediate 9728,
 # 32 q / 8 kv heads x 128) and 14B-like (hidden 5120, intermediate 17408,
 # 40 q / 8 kv heads x 128); QKV and gate+up fused.

@@ -61,7 +61,7 @@ def call_bytes(T, n_in, n_out):
 # projections (qkv 13.24 MB, o 8.88 MB, gate+up 61.18 MB, down 31.00 MB), from
 # one ncu capture of the current kernel at 16 tokens; the command is in
 # profiles/gemv_kernel_gate_up_4096x28672_t16.md. None once the kernel changes.
-GEMV_TRAFFIC_PER_LAUNCH_T16 = (13236736 + 8878336 + 61178624 + 31001344) / 4
+GEMV_TRAFFIC_PER_LAUNCH_T16 = (13237248 + 8878592 + 61182464 + 30997248) / 4
 
 
 def peaks():

@@ -128,12 +128,12 @@ struct Zero2 {
     uint32_t zb0, zc0, zb1, zc1;
 };
 __device__ __forceinline__ Zero2 zero_consts(uint32_t zbyte) {
-    const uint32_t z0 = zbyte & 0xFu, z1 = (zbyte >> 4) & 0xFu;
+    const uint32_t t = __byte_perm(zbyte, 0u, 0x4040);     // the byte at bits 0-7 and 16-23
     Zero2 r;
-    r.zb0 = (0x6400u | z0) * 0x00010001u;
-    r.zb1 = (0x6400u | z1) * 0x00010001u;
-    r.zc0 = (0xD400u | (z0 << 4)) * 0x00010001u;
-    r.zc1 = (0xD400u | (z1 << 4)) * 0x00010001u;
+    r.zb0 = lop3_and_or(t, 0x000F000Fu, 0x64006400u);
+    r.zb1 = lop3_and_or(t >> 4, 0x000F000Fu, 0x64006400u);
+    r.zc0 = lop3_and_or(t << 4, 0x00F000F0u, 0xD400D400u);
+    r.zc1 = lop3_and_or(t, 0x00F000F0u, 0xD400D400u);
     return r;
 }
 

@@ -62,6 +62,7 @@ struct GemvArgs {
     const uint8_t* zp;
     const __half* bias;   // [out] fp16 or null
     __half* Y;
+    int xlm;              // X' already lane-major within 64-channel blocks
 };
 
 // Not volatile: the MMA reads registers only, so the compiler may schedule
@@ -202,18 +203,26 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         // >= T are zero-filled by a source size of 0), then one wait. Within
         // each 64-channel block the row is stored lane-major: channel
         // 16 j + 4 q + e at position 16 q + 4 j + e, so lane q of a fragment
-        // row finds the four k tiles' B values in 32 contiguous bytes.
-        const int pieces_per_row = ncg * 32;                // 8-byte pieces of 4 channels
-        const int total = NT * 8 * pieces_per_row;
-        const __half* xsrc = a.Xr + (size_t)g_begin * 128;
-        for (int i = threadIdx.x; i < total; i += kWarps * 32) {
-            const int tok = i / pieces_per_row, v = i - tok * pieces_per_row;   // v: 4-channel piece
-            const int blk = v >> 4, jq = v & 15, j = jq >> 2, q = jq & 3;       // channel 64 blk + 16 j + 4 q
-            const bool real = tok < a.T;
-            const __half* src = xsrc + (size_t)(real ? tok : 0) * a.in + 4 * v;
-            const uint32_t dst = smem_u32(xs + (size_t)tok * XS + blk * 64 + 16 * q + 4 * j);
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(real ? 8 : 0)
-                         : "memory");
+        // row finds the four k tiles' B values in 32 contiguous bytes. Warp w
+        // copies token row w mod 8 NT (two warps per row when NT == 1).
+        constexpr int kRows = NT * 8, kParts = kWarps / kRows;
+        const int tok = warp & (kRows - 1), part = warp / kRows;
+        const bool real = tok < a.T;
+        const unsigned char* srow =
+            reinterpret_cast<const unsigned char*>(a.Xr + (size_t)(real ? tok : 0) * a.in + (size_t)g_begin * 128);
+        const uint32_t drow = smem_u32(xs + (size_t)tok * XS);
+        if (a.xlm) {                                       // the rotation wrote that order: a plain copy
+            const int n16 = ncg * 16;
+            for (int v = part * 32 + lane; v < n16; v += 32 * kParts)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(drow + 16 * v), "l"(srow + 16 * v),
+                             "r"(real ? 16 : 0) : "memory");
+        } else {                                           // natural order: 8-byte pieces of 4 channels
+            const int n8 = ncg * 32;
+            for (int v = part * 32 + lane; v < n8; v += 32 * kParts) {
+                const int blk = v >> 4, j = (v >> 2) & 3, q = v & 3;   // channel 64 blk + 16 j + 4 q
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(drow + 2 * (blk * 64 + 16 * q + 4 * j)),
+                             "l"(srow + 8 * v), "r"(real ? 8 : 0) : "memory");
+            }
         }
         cp_async_commit();
         for (int i = threadIdx.x; i < NT * 8 * SR; i += kWarps * 32) red[i] = 0.f;
@@ -509,7 +518,7 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     const int K = rot ? rot->K : 0;
     const void* xr = X;
     if (rot) {
-        cudaError_t e = launch_rotate_decode(*rot, X, ws, T, s);
+        cudaError_t e = launch_rotate_decode(*rot, X, ws, T, s, true);
         if (e != cudaSuccess) return e;
         xr = ws;
     }
@@ -530,6 +539,7 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.zp = static_cast<const uint8_t*>(zp);
     a.bias = static_cast<const __half*>(bias);
     a.Y = static_cast<__half*>(Y);
+    a.xlm = rot ? 1 : 0;
     cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, s) : launch_gemv_t<1>(a, p, s);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

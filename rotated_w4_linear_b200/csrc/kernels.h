@@ -21,7 +21,10 @@ struct RotDev {
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
 // Decode batches (1 <= T <= 16): one CTA per group, all layers' parameters in
 // shared memory; launched as a programmatic dependent of the previous kernel.
-cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
+// lane_major: X' is written with every 64-channel block in the decode
+// kernel's B-fragment order (channel 16 j + 4 q + e at 16 q + 4 j + e).
+cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s,
+                                 bool lane_major = false);
 size_t rotate_decode_smem(int K, int T);
 
 cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out,

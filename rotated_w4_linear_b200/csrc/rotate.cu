@@ -127,11 +127,14 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
 // exchange buffers alternately (one warp barrier per quad and layer) and
 // loads the next item's X while it rotates the current one. The operations
 // and their order are those of rotate_kernel, so X' is bit-identical.
+// lane_major != 0 writes each 64-channel block of X' in the order the decode
+// kernel's B fragments read it: channel 16 j + 4 q + e at position
+// 16 q + 4 j + e (the values are the same, only their places change).
 template <int QW>
 __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restrict__ X, __half* __restrict__ Xr,
                                                           int T, int in, int G, int K,
                                                           const uint8_t* __restrict__ rotq,
-                                                          const float* __restrict__ inv_alpha) {
+                                                          const float* __restrict__ inv_alpha, int lane_major) {
     constexpr int NBUF = QW > 1 ? 2 : 1;
     asm volatile("griddepcontrol.launch_dependents;");
     extern __shared__ __align__(16) unsigned char sm[];
@@ -251,7 +254,10 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
                 }
             }
         }
-        const int t0 = tile * tile_tokens + warp * 4 * QW, c0 = g * 128 + 4 * lane;
+        const int t0 = tile * tile_tokens + warp * 4 * QW;
+        // lane L holds channels 4L..4L+3 = 64 b + 16 j + 4 q + (0..3) with L = 16 b + 4 j + q
+        const int piece = lane_major ? ((lane & 16) | ((lane & 3) << 2) | ((lane >> 2) & 3)) : lane;
+        const int c0 = g * 128 + 4 * piece;
 #pragma unroll
         for (int q = 0; q < QW; ++q) {
 #pragma unroll
@@ -277,7 +283,8 @@ namespace {
 constexpr int QW_BIG = 2;
 
 template <int QW>
-cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int warps, cudaStream_t s) {
+cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int warps, cudaStream_t s,
+                        int lane_major) {
     constexpr int NBUF = QW > 1 ? 2 : 1;
     const size_t smem = (size_t)r.K * kRotQBlockBytes + (size_t)warps * 2048 * NBUF;
     if (smem > 48 * 1024) {
@@ -306,7 +313,7 @@ cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_quad_kernel<QW>, static_cast<const __half*>(X),
                                              static_cast<__half*>(Xr), (int)T, (int)r.in, r.G, r.K,
-                                             (const uint8_t*)r.rotq, (const float*)r.inv_alpha);
+                                             (const uint8_t*)r.rotq, (const float*)r.inv_alpha, lane_major);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -314,10 +321,11 @@ cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int
 
 size_t rotate_decode_smem(int K, int T) { return (size_t)K * kRotQBlockBytes + (size_t)((T + 3) / 4) * 2048; }
 
-cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s) {
+cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s,
+                                 bool lane_major) {
     if (T <= 0) return cudaSuccess;
     if (T > 16) return cudaErrorInvalidValue;
-    return launch_quad<1>(r, X, Xr, T, (int)((T + 3) / 4), s);
+    return launch_quad<1>(r, X, Xr, T, (int)((T + 3) / 4), s, lane_major ? 1 : 0);
 }
 
 template <int TT>
@@ -341,7 +349,7 @@ cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, c
     const __half* x = static_cast<const __half*>(X);
     __half* y = static_cast<__half*>(Xr);
     if (T <= 16) return launch_rotate_decode(r, X, Xr, T, s);
-    if (T >= 256) return launch_quad<QW_BIG>(r, X, Xr, T, 8, s);
+    if (T >= 256) return launch_quad<QW_BIG>(r, X, Xr, T, 8, s, 0);
     const cudaError_t e = launch_rotate_t<8>(r, x, y, T, s);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

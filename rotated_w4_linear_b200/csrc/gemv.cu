@@ -9,9 +9,11 @@
 // and waits (griddepcontrol.wait) before it reads X'. It lets the next
 // kernel launch early in turn.
 //
-//   work split: the CTA's items (one row block of 16 rows x two groups: 2 KB
-//     of int4 codes + scales + zeros) in row-block-major order are cut into
-//     sixteen equal contiguous runs, one per warp;
+//   work split: the CTA's (row block of 16 rows, 128-channel group) units in
+//     row-block-major order are cut into sixteen contiguous runs that differ
+//     by at most one unit, one per warp; a warp walks its run in items of up
+//     to two groups (2 KB of int4 codes + scales + zeros) that stay inside
+//     one row block;
 //   weight stream: each warp streams its run through a private 3-stage
 //     shared-memory ring with cp.async (16-byte global->shared copies that
 //     bypass the registers): one commit group per item, wait on the oldest,
@@ -77,11 +79,17 @@ __device__ __forceinline__ void mma16816(float c[4], const uint32_t a[4], uint32
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// 16-byte global -> shared copies (bypassing L1) under a predicate that is
+// evaluated inside the asm, so a condition costs one setp instead of a
+// divergent branch around the copy.
+__device__ __forceinline__ void cp_async16_if(bool pred, uint32_t dst, const void* src) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}"
+                 ::"r"(dst), "l"(src), "r"((int)pred) : "memory");
 }
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+// 8 bytes, 8-byte aligned, through L1
+__device__ __forceinline__ void cp_async8_if(bool pred, uint32_t dst, const void* src) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p cp.async.ca.shared.global [%0], [%1], 8;\n\t}"
+                 ::"r"(dst), "l"(src), "r"((int)pred) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -104,8 +112,8 @@ __device__ __forceinline__ void cluster_sync() {
 
 // A lane's source pointers for the items of one row block: codes (the
 // lane's 16 bytes of each 512-byte k block), scales (lanes 0..3: 16 bytes
-// each) and zeros (lane 31: the item's 16 bytes). Within a row block the
-// next item is 2 KB, 64 B and 16 B further on.
+// each) and zeros (lanes 30, 31: 8 bytes per group). Within a row block the
+// next group is 1 KB, 32 B and 8 B further on.
 struct ItemSrc {
     const uint4* q;
     const uint32_t* sc;
@@ -123,15 +131,16 @@ __device__ __forceinline__ ItemSrc item_src(const GemvArgs& a, int rb, int g0, i
 
 // Copy one item (groups g0, g0+1 if ng == 2 of the source's row block) into
 // a ring slot; `dst` is the slot address plus this lane's 16-byte offset.
+// Slot layout: codes [2 ng][512 B], scales [ng][32 B] at kItemQBytes, zeros
+// [ng][8 B] after the scales of kItemGroups groups.
 __device__ __forceinline__ void issue_item(const ItemSrc& p, uint32_t slot, uint32_t dst, int ng, int lane) {
 #pragma unroll
-    for (int kb = 0; kb < 2 * kItemGroups; ++kb)
-        if (kb < 2 * ng) cp_async16(dst + kb * 512, p.q + kb * 32);
-    if (lane < 2 * ng) cp_async16(slot + kItemQBytes + lane * 16, p.sc);
-    if (lane == 31) {
-        if (ng == 2) cp_async16(slot + kItemQBytes + kItemGroups * 32, p.z);
-        else cp_async8(slot + kItemQBytes + kItemGroups * 32, p.z);
-    }
+    for (int kb = 0; kb < 2 * kItemGroups; ++kb) cp_async16_if(kb < 2 * ng, dst + kb * 512, p.q + kb * 32);
+    cp_async16_if(lane < 2 * ng, slot + kItemQBytes + lane * 16, p.sc);
+    // zeros: 8 bytes per group from lanes 30 and 31 (an item may start at an
+    // odd group, so the pair need not be 16-byte aligned)
+    const int zg = lane & 1;
+    cp_async8_if(lane >= 32 - kItemGroups && zg < ng, slot + kItemQBytes + kItemGroups * 32 + 8 * zg, p.z + 8 * zg);
 }
 
 }  // namespace
@@ -152,15 +161,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     const int g_begin = chunk * a.KC;
     const int g_end = min(a.G, g_begin + a.KC);
     const int ncg = max(0, g_end - g_begin);
-    const int nsub = (ncg + kItemGroups - 1) / kItemGroups;
     const int nrb = a.out >> 4;
     const int rb_begin = rt * a.RT;
     const int nrbt = max(0, min(nrb, rb_begin + a.RT) - rb_begin);
-    // items (row block, sub) in row-block-major order; warp w takes the
-    // contiguous run [items*w/8, items*(w+1)/8)
-    const int items = nrbt * nsub;
-    const int i_lo = (int)(((int64_t)items * warp) / kWarps);
-    const int nmine = (int)(((int64_t)items * (warp + 1)) / kWarps) - i_lo;
+    // The CTA's (row block, group) units in row-block-major order, flattened
+    // as f = (rb - rb_begin) ncg + (g - g_begin); warp w takes the contiguous
+    // run [F w / 16, F (w + 1) / 16) of the F units (runs differ by at most
+    // one group) and walks it in items of up to two groups that end at a row
+    // block's last group or at the run's end.
+    const int F = nrbt * ncg;
+    const int f_lo = (int)(((int64_t)F * warp) / kWarps);
+    const int f_hi = (int)(((int64_t)F * (warp + 1)) / kWarps);
+    const int rbl_lo = ncg ? f_lo / ncg : 0;                // first row block (tile-local) and group
+    const int g_lo = g_begin + (ncg ? f_lo - rbl_lo * ncg : 0);
 
     const int XS = a.KC * 128 + 8;                         // halves; row stride == 16 bytes mod 128
     const int SR = a.RT * 16 + 4;                          // floats per token row of the partial tile
@@ -169,22 +182,24 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     unsigned char* ring = reinterpret_cast<unsigned char*>(red + NT * 8 * SR);
     const uint32_t ring_w = smem_u32(ring) + (uint32_t)(warp * kStages * kItemBytes);
 
-    // producer cursor: (row block, sub) of the next item to copy and the
-    // lane's source pointers, advanced incrementally
-    int p_rb = rb_begin + (nsub ? i_lo / nsub : 0), p_sub = nsub ? i_lo % nsub : 0;
-    ItemSrc src = item_src(a, p_rb, g_begin + p_sub * kItemGroups, lane);
+    // producer cursor: position, row block and group of the next item to
+    // copy and the lane's source pointers, advanced incrementally
+    int p_f = f_lo, p_rb = rb_begin + rbl_lo, p_g = g_lo;
+    ItemSrc src = item_src(a, p_rb, p_g, lane);
     auto issue_next = [&](int stage) {
-        const int g0 = g_begin + p_sub * kItemGroups;
+        const int ng = min(min(kItemGroups, g_end - p_g), f_hi - p_f);
         const uint32_t slot = ring_w + stage * kItemBytes;
-        issue_item(src, slot, slot + lane * 16, min(kItemGroups, g_end - g0), lane);
-        if (++p_sub == nsub) {
-            p_sub = 0;
+        issue_item(src, slot, slot + lane * 16, ng, lane);
+        p_f += ng;
+        p_g += ng;
+        if (p_g == g_end) {
+            p_g = g_begin;
             ++p_rb;
             src = item_src(a, p_rb, g_begin, lane);
         } else {
-            src.q += kItemGroups * 2 * 32;
-            src.sc += kItemGroups * 8;
-            src.z += kItemGroups * 8;
+            src.q += ng * 2 * 32;
+            src.sc += ng * 8;
+            src.z += ng * 8;
         }
     };
 
@@ -192,7 +207,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     // are never written by the kernels this one may overlap)
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
-        if (s < nmine) issue_next(s);
+        if (p_f < f_hi) issue_next(s);
         cp_async_commit();
     }
 
@@ -260,18 +275,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
             for (int c = 0; c < 2; ++c) acc[nt][c][0] = acc[nt][c][1] = acc[nt][c][2] = acc[nt][c][3] = 0.f;
         }
     };
-    int c_rbl = nsub ? i_lo / nsub : 0, c_sub = nsub ? i_lo % nsub : 0;   // item being consumed
+    int c_f = f_lo, c_rbl = rbl_lo, c_g = g_lo;            // item being consumed
+    bool pending = false;                                  // sums not yet flushed
     int stage = 0, pstage = kStages - 1;
-    for (int i = 0; i < nmine; ++i) {
-        if (i + kStages - 1 < nmine) issue_next(pstage);
+    while (c_f < f_hi) {
+        if (p_f < f_hi) issue_next(pstage);
         cp_async_commit();
         pstage = (pstage + 1 == kStages) ? 0 : pstage + 1;
         cp_async_wait<kStages - 1>();
         __syncwarp();
 
         const unsigned char* slot = ring_p + stage * kItemBytes;
-        const int ng = min(kItemGroups, ncg - c_sub * kItemGroups);
-        const int kb_off = c_sub * kItemGroups * 128 * 2;  // bytes into the X' rows
+        const int ng = min(min(kItemGroups, g_end - c_g), f_hi - c_f);   // as the producer chose
+        const int kb_off = (c_g - g_begin) * 128 * 2;      // bytes into the X' rows
 #pragma unroll
         for (int g = 0; g < kItemGroups; ++g) {
             if (g < ng) {
@@ -306,13 +322,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         }
         __syncwarp();                                      // the slot may be refilled from here on
         stage = (stage + 1 == kStages) ? 0 : stage + 1;
-        if (++c_sub == nsub) {                             // row block done
+        c_f += ng;
+        c_g += ng;
+        pending = true;
+        if (c_g == g_end) {                                // row block done
             flush(c_rbl);
-            c_sub = 0;
+            pending = false;
+            c_g = g_begin;
             ++c_rbl;
         }
     }
-    if (nmine > 0 && c_sub != 0) flush(c_rbl);             // run ended inside a row block
+    if (pending) flush(c_rbl);                             // run ended inside a row block
     if (NT == 2) asm volatile("griddepcontrol.launch_dependents;");
     cp_async_wait<0>();
     __syncthreads();
@@ -431,7 +451,6 @@ GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
         if (KC > kc_max) continue;
         const int ns = (G + KC - 1) / KC;
         if (ns != nsplit) continue;
-        const int nsub = (KC + kItemGroups - 1) / kItemGroups;
         for (int RT = 1; RT <= std::min(nrb, 64); ++RT) {
             const size_t smem = gemv_smem(NT, KC, RT);
             if (smem > 200 * 1024) break;
@@ -444,7 +463,8 @@ GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
             const int rowtiles = (nrb + RT - 1) / RT;
             const int ctas = ns * rowtiles;
             const int waves = (ctas + slots - 1) / slots;
-            const double per_warp = std::ceil((double)RT * nsub / kWarps);
+            // items per warp: runs of ceil(RT KC / 16) groups in items of two
+            const double per_warp = std::ceil((double)RT * KC / kWarps) / kItemGroups;
             // +3: pipeline fill and epilogue per CTA; a partly empty wave
             // still costs its share of HBM time
             const double fill = (double)ctas / ((double)waves * slots);

@@ -212,6 +212,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     }
 
     // ---- X' chunk and partial tile (waits for the previous grid: X' may be its output)
+    // Unrotated calls: L2 prefetch of the X chunk (one 128-byte line per
+    // thread and pass). A prefetch returns no data, so it may run before the
+    // wait even if X is the previous grid's output; it saves the DRAM latency
+    // when X is not in L2. (A rotated X' was just written by the rotation
+    // kernel and sits in L2.)
+    if (!a.xlm)
+        for (int i = threadIdx.x; i < NT * 8 * 2 * ncg; i += kWarps * 32) {
+            const int tok = i / (2 * ncg), l = i - tok * 2 * ncg;
+            if (tok < a.T)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.Xr + (size_t)tok * a.in + (size_t)g_begin * 128 + l * 64));
+        }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
         // all of the chunk's copies are in flight at once (cp.async; rows

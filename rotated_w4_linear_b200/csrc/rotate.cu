@@ -158,6 +158,16 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
     };
     int cur_g = (int)(w_lo / ntiles);
     copy_tables(cur_g);
+    {
+        // Ask L2 for the first item's X rows (two 128-byte lines per token)
+        // while the previous grid finishes. A prefetch returns no data, so it
+        // is safe even when X is that grid's output: the loads below still
+        // come after the wait and read what the grid wrote.
+        const int tile = (int)(w_lo - (int64_t)cur_g * ntiles);
+        const int t = tile * tile_tokens + warp * 4 * QW + (lane >> 1);
+        if (lane < 8 * QW && t < T)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(X + (size_t)t * in + cur_g * 128 + (lane & 1) * 64));
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");   // X may be the previous grid's output
 
     uint2 raw[QW][4];                                      // X of the item to rotate next, fp16

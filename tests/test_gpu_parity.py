@@ -192,7 +192,7 @@ def _layer(B, in_f, out_f, K, P, seed, oracle_quant=True):
     (40, 384, 48, 8, 64),      # partial 128-row tile, odd group count
     (130, 512, 256, 8, 64),    # two 128-token tiles, ragged
     (300, 256, 160, 4, 13),    # 256-token tiles, ragged rows and tokens
-    (2500, 384, 96, 8, 64),    # rotation in token chunks overlapped with the GEMM, ragged last chunk
+    (2500, 384, 96, 8, 64),    # twenty 128-token tiles, ragged last tile
 ])
 def test_linear_parity_exhaustive(B, T, in_f, out_f, K, P):
     seed = synth.layer_seed(0, T * 7 + K)

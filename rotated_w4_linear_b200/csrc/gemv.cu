@@ -149,11 +149,13 @@ template <int NT>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) {
     // When the next kernel on the stream may launch (it prefetches only its
     // weights, or its tables, before it waits for this grid to complete):
-    // at 8 tokens or fewer right away; above that after the mainloop, so that
-    // the next rotation kernel's CTAs land on SMs as this grid's CTAs leave
-    // instead of crowding the few SMs this grid left free (measured: the
-    // early trigger costs 1.5-2 us per projection at 16 tokens, the late one
-    // 0.5-1 us at 1 token).
+    // at 8 tokens or fewer right away; above that once every warp of the CTA
+    // has at most one item left, so that the next rotation kernel's CTAs land
+    // on SMs as this grid's CTAs leave instead of crowding the few SMs this
+    // grid left free (measured at 12 and 16 tokens: the trigger at the start
+    // costs about 2 us per layer of four projections, the one after the
+    // mainloop about 0.6 us more than this one; at 1 token the late trigger
+    // costs 0.5-1 us per projection). Warps without work trigger at the end.
     if (NT == 1) asm volatile("griddepcontrol.launch_dependents;");
     extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -288,6 +290,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     };
     int c_f = f_lo, c_rbl = rbl_lo, c_g = g_lo;            // item being consumed
     bool pending = false;                                  // sums not yet flushed
+    bool trig = false;
     int stage = 0, pstage = kStages - 1;
     while (c_f < f_hi) {
         if (p_f < f_hi) issue_next(pstage);
@@ -336,6 +339,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         c_f += ng;
         c_g += ng;
         pending = true;
+        if (NT == 2 && !trig && f_hi - c_f <= kItemGroups) {   // one item left at most
+            asm volatile("griddepcontrol.launch_dependents;");
+            trig = true;
+        }
         if (c_g == g_end) {                                // row block done
             flush(c_rbl);
             pending = false;

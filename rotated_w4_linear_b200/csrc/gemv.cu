@@ -109,6 +109,13 @@ __device__ __forceinline__ float4 ld_dsmem4(uint32_t addr) {   // 16-byte aligne
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Cluster barrier without memory ordering: for the last barrier, which only
+// keeps each CTA's shared memory alive until the other CTAs' reads of it are
+// done (their values are already used). A release here would also wait for
+// this CTA's global stores of Y to complete, about a microsecond.
+__device__ __forceinline__ void cluster_sync_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
 
 // A lane's source pointers for the items of one row block: codes (the
 // lane's 16 bytes of each 512-byte k block), scales (lanes 0..3: 16 bytes
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         *reinterpret_cast<uint2*>(a.Y + (size_t)t * a.out + row0 + r) =
             make_uint2(pack_half2(sum.x, sum.y), pack_half2(sum.z, sum.w));
     }
-    cluster_sync();                                        // tiles stay alive until every reader is done
+    cluster_sync_relaxed();                                // tiles stay alive until every reader is done
 }
 
 namespace {

@@ -127,10 +127,11 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
 // exchange buffers alternately (one warp barrier per quad and layer) and
 // loads the next item's X while it rotates the current one. The operations
 // and their order are those of rotate_kernel, so X' is bit-identical.
+// PF: each layer's table entries are loaded during the layer before.
 // lane_major != 0 writes each 64-channel block of X' in the order the decode
 // kernel's B fragments read it: channel 16 j + 4 q + e at position
 // 16 q + 4 j + e (the values are the same, only their places change).
-template <int QW>
+template <int QW, bool PF>
 __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restrict__ X, __half* __restrict__ Xr,
                                                           int T, int in, int G, int K,
                                                           const uint8_t* __restrict__ rotq,
@@ -218,11 +219,31 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
             }
         }
         if (QW > 1 && w + 1 < w_hi) load_item(w + 1);     // in flight during the layers
+        // With PF, layer t's positions and coefficients are loaded during
+        // layer t - 1 (the exchange's asm statements are compiler barriers,
+        // so the loads are placed by hand before them), which takes their
+        // latency off the chain store -> barrier -> load -> fma of a layer.
+        uint2 pos = make_uint2(0u, 0u);
+        float4 c01 = make_float4(0.f, 0.f, 0.f, 0.f), c23 = c01;
+        if (PF && K > 0) {
+            pos = *reinterpret_cast<const uint2*>(prm + 8 * lane);
+            c01 = *reinterpret_cast<const float4*>(prm + 256 + 16 * lane);
+            c23 = *reinterpret_cast<const float4*>(prm + 768 + 16 * lane);
+        }
         for (int t = 0; t < K; ++t) {
             const unsigned char* blk = prm + (size_t)t * kRotQBlockBytes;
-            const uint2 pos = *reinterpret_cast<const uint2*>(blk + 8 * lane);
-            const float4 c01 = *reinterpret_cast<const float4*>(blk + 256 + 16 * lane);
-            const float4 c23 = *reinterpret_cast<const float4*>(blk + 768 + 16 * lane);
+            if (!PF) {
+                pos = *reinterpret_cast<const uint2*>(blk + 8 * lane);
+                c01 = *reinterpret_cast<const float4*>(blk + 256 + 16 * lane);
+                c23 = *reinterpret_cast<const float4*>(blk + 768 + 16 * lane);
+            }
+            uint2 pos_n = pos;
+            float4 c01_n = c01, c23_n = c23;
+            if (PF && t + 1 < K) {
+                pos_n = *reinterpret_cast<const uint2*>(blk + kRotQBlockBytes + 8 * lane);
+                c01_n = *reinterpret_cast<const float4*>(blk + kRotQBlockBytes + 256 + 16 * lane);
+                c23_n = *reinterpret_cast<const float4*>(blk + kRotQBlockBytes + 768 + 16 * lane);
+            }
             const float ca[4] = {c01.x, c01.z, c23.x, c23.z}, cb[4] = {c01.y, c01.w, c23.y, c23.w};
             uint32_t st[4], ld[4];
             bool act[4];                                   // channel in a pair of this layer
@@ -263,6 +284,9 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
                     for (int h = 0; h < 2; ++h) v[q][j][h] = f2_fma(b2, p[j][h], f2_mul(a2, v[q][j][h]));
                 }
             }
+            pos = pos_n;
+            c01 = c01_n;
+            c23 = c23_n;
         }
         const int t0 = tile * tile_tokens + warp * 4 * QW;
         // lane L holds channels 4L..4L+3 = 64 b + 16 j + 4 q + (0..3) with L = 16 b + 4 j + q
@@ -292,14 +316,14 @@ namespace {
 // larger batches: 8 warps of QW_BIG quads (4 QW_BIG tokens) per CTA
 constexpr int QW_BIG = 2;
 
-template <int QW>
+template <int QW, bool PF>
 cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int warps, cudaStream_t s,
                         int lane_major) {
     constexpr int NBUF = QW > 1 ? 2 : 1;
     const size_t smem = (size_t)r.K * kRotQBlockBytes + (size_t)warps * 2048 * NBUF;
     if (smem > 48 * 1024) {
         const cudaError_t e =
-            cudaFuncSetAttribute(rotate_quad_kernel<QW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            cudaFuncSetAttribute(rotate_quad_kernel<QW, PF>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     const int64_t ntiles = (T + (int64_t)warps * 4 * QW - 1) / ((int64_t)warps * 4 * QW);
@@ -308,7 +332,7 @@ cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int
         int dev = 0, sms = 148, per_sm = 1;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quad_kernel<QW>, 32 * warps, smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quad_kernel<QW, PF>, 32 * warps, smem);
         ctas = std::min<int64_t>(ctas, (int64_t)sms * std::max(per_sm, 1));
     }
     cudaLaunchConfig_t cfg{};
@@ -321,7 +345,7 @@ cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_quad_kernel<QW>, static_cast<const __half*>(X),
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_quad_kernel<QW, PF>, static_cast<const __half*>(X),
                                              static_cast<__half*>(Xr), (int)T, (int)r.in, r.G, r.K,
                                              (const uint8_t*)r.rotq, (const float*)r.inv_alpha, lane_major);
     return e != cudaSuccess ? e : cudaGetLastError();
@@ -335,7 +359,11 @@ cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64
                                  bool lane_major) {
     if (T <= 0) return cudaSuccess;
     if (T > 16) return cudaErrorInvalidValue;
-    return launch_quad<1>(r, X, Xr, T, (int)((T + 3) / 4), s, lane_major ? 1 : 0);
+    // prefetching the next layer's tables pays with several warps per CTA
+    // (measured: 2% of the decode step at 16 tokens) but not with one or two
+    const int warps = (int)((T + 3) / 4);
+    return T > 8 ? launch_quad<1, true>(r, X, Xr, T, warps, s, lane_major ? 1 : 0)
+                 : launch_quad<1, false>(r, X, Xr, T, warps, s, lane_major ? 1 : 0);
 }
 
 template <int TT>
@@ -359,7 +387,7 @@ cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, c
     const __half* x = static_cast<const __half*>(X);
     __half* y = static_cast<__half*>(Xr);
     if (T <= 16) return launch_rotate_decode(r, X, Xr, T, s);
-    if (T >= 256) return launch_quad<QW_BIG>(r, X, Xr, T, 8, s, 0);
+    if (T >= 256) return launch_quad<QW_BIG, true>(r, X, Xr, T, 8, s, 0);
     const cudaError_t e = launch_rotate_t<8>(r, x, y, T, s);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -58,10 +58,10 @@ def call_bytes(T, n_in, n_out):
 
 
 # DRAM bytes (read + write) per decode-kernel launch, mean over the four
-# projections (qkv 13.24 MB, o 8.88 MB, gate+up 61.18 MB, down 31.00 MB), from
+# projections (qkv 13.24 MB, o 8.89 MB, gate+up 61.18 MB, down 31.00 MB), from
 # one ncu capture of the current kernel at 16 tokens; the command is in
 # profiles/gemv_kernel_gate_up_4096x28672_t16.md. None once the kernel changes.
-GEMV_TRAFFIC_PER_LAUNCH_T16 = (13237248 + 8878592 + 61182464 + 30997248) / 4
+GEMV_TRAFFIC_PER_LAUNCH_T16 = (13238528 + 8886272 + 61180416 + 30999040) / 4
 
 
 def peaks():
@@ -334,14 +334,15 @@ def bench_prefill(args, torch, B, local):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     times = {}
-    for rot in (True, False):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            graphs[rot].replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        times[rot] = e0.elapsed_time(e1) / 1e3 / args.steps
+    with ClockSampler(local) as clk:
+        for rot in (True, False):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                graphs[rot].replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times[rot] = e0.elapsed_time(e1) / 1e3 / args.steps
     flops = sum(2.0 * T * p["n_in"] * p["n_out"] for p in calls)
     _, _, kind = peaks()
     try:
@@ -356,7 +357,8 @@ def bench_prefill(args, torch, B, local):
                       "rotation_overhead": times[True] / times[False] - 1.0,
                       "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
                                    "frac": tf / tc_peak, "peak_source": f"{kind} bf16_tflops_sustained "
-                                   "(fp16 and bf16 share the dense tensor rate)"}}), flush=True)
+                                   "(fp16 and bf16 share the dense tensor rate)"},
+                      "clocks": clk.summary()}), flush=True)
     del graphs
     for p in calls:
         p["rot"].close()

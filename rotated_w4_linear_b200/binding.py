@@ -67,9 +67,18 @@ def _check(fn: str, st: int) -> None:
         raise ParoError(fn, st, lib().paro_last_error().decode())
 
 
-def _stream(stream) -> int:
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, device: Optional[torch.device] = None) -> int:
+    """Raw cudaStream_t: the given stream, else the current stream of the
+    tensor's device (read without building a torch Stream object, which
+    costs a few microseconds per call on the decode path)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        idx = device.index if device is not None and device.index is not None else torch.cuda.current_device()
+        if _raw_stream is not None:
+            return int(_raw_stream(idx))
+        stream = torch.cuda.current_stream(idx)
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
@@ -122,7 +131,7 @@ def paro_rotate(rot: Rotation, X: torch.Tensor, Xr: Optional[torch.Tensor] = Non
     _dev(X, torch.float16, "X"), _dev(Xr, torch.float16, "Xr")
     if X.shape != Xr.shape or X.dim() != 2 or X.shape[1] != rot.in_features:
         raise ValueError("X/Xr must be [tokens][in_features]")
-    _check("paro_rotate", lib().paro_rotate(rot.handle, X.data_ptr(), Xr.data_ptr(), X.shape[0], _stream(stream)))
+    _check("paro_rotate", lib().paro_rotate(rot.handle, X.data_ptr(), Xr.data_ptr(), X.shape[0], _stream(stream, X.device)))
     return Xr
 
 
@@ -197,7 +206,7 @@ def paro_linear(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_featur
         rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
         _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"),
         _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
-        _stream(stream)))
+        _stream(stream, X.device)))
     return Y
 
 
@@ -219,7 +228,7 @@ def paro_linear_bias(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, bias:
         rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
         _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"), b,
         _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
-        _stream(stream)))
+        _stream(stream, X.device)))
     return Y
 
 
@@ -233,5 +242,5 @@ def paro_linear_noalloc(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, ou
     _check("paro_linear_noalloc", lib().paro_linear_noalloc(
         rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
         _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"),
-        _dev(Y, torch.float16, "Y"), T, in_f, out_features, _stream(stream)))
+        _dev(Y, torch.float16, "Y"), T, in_f, out_features, _stream(stream, X.device)))
     return Y

@@ -89,14 +89,15 @@ def test_rotate_parity(B, T, in_f, K, P):
 @pytest.mark.parametrize("in_f,K,P", [(4096, 8, 64), (14336, 16, 13), (384, 3, 64)])
 def test_rotate_kernels_agree_bit_for_bit(B, in_f, K, P):
     """Batches of at most 16 tokens and of 256 or more take the quad kernel
-    (float4 exchange, packed f32x2 arithmetic); the others the general one.
-    All apply the same operations in the same order: identical bits."""
+    (float4 exchange, packed f32x2 arithmetic; from 9 tokens on with each
+    layer's tables loaded during the layer before); the others the general
+    one. All apply the same operations in the same order: identical bits."""
     seed = synth.layer_seed(1, 77 + K)
     pairs, theta, alpha = synth.rotation_params(in_f, K, seed, pairs_per_group=P)
     x = synth.activations(24, in_f, seed)
     rot = B.paro_rot_create(pairs, theta, alpha)
     big = host(B.paro_rotate(rot, dev(x)))
-    for T in (1, 7, 16):
+    for T in (1, 7, 8, 9, 16):
         small = host(B.paro_rotate(rot, dev(x[:T])))
         assert np.array_equal(small.view(np.uint16), big[:T].view(np.uint16)), T
     check_rotation(big[:16], x[:16], pairs, theta, alpha)

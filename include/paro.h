@@ -44,7 +44,7 @@ extern "C" {
 typedef enum {
     PARO_OK = 0,
     PARO_ERR_ARG = 1,          /* invalid argument (null, size, alignment, pair table) */
-    PARO_ERR_UNSUPPORTED = 2,  /* valid but not supported by this build (e.g. group != 128) */
+    PARO_ERR_UNSUPPORTED = 2,  /* valid but not supported by this library (e.g. group != 128) */
     PARO_ERR_CUDA = 3,         /* a CUDA runtime call or a kernel launch failed */
     PARO_ERR_DEVICE = 4        /* no usable sm_100 device */
 } paro_status;

@@ -22,7 +22,7 @@ Orientation: the pages write Y = X W with W of shape [in][out]; T acts on the
 input channels (rows of that W). Here weights are stored [out][in] (PyTorch
 orientation), so T acts along the last axis of every output row.
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
   * product order: layer t = 1 is applied first after diag(alpha), i.e.
     T = R_K ... R_1 diag(alpha) (the CSDN pseudo-code scales first, then
     rotates in list order);

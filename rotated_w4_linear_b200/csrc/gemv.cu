@@ -491,9 +491,13 @@ GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
             // items per warp: runs of ceil(RT KC / 16) groups in items of two
             const double per_warp = std::ceil((double)RT * KC / kWarps) / kItemGroups;
             // +3: pipeline fill and epilogue per CTA; a partly empty wave
-            // still costs its share of HBM time
+            // still costs its share of HBM time; a split-k cluster adds its
+            // barrier and distributed-shared-memory reduction, measured at
+            // about 1.5 items' time (plan sweeps of Qwen3- and Llama-shaped
+            // layers at 1 and 8 tokens)
             const double fill = (double)ctas / ((double)waves * slots);
-            const double cost = waves * (per_warp + 3.0) * (1.0 + 0.3 * (1.0 - fill)) + 0.05 * ns;
+            const double cost = waves * (per_warp + 3.0) * (1.0 + 0.3 * (1.0 - fill)) + 0.05 * ns +
+                                (ns > 1 ? 1.5 : 0.0);
             if (cost < best_cost - 1e-9) {
                 best_cost = cost;
                 best.KC = KC;

@@ -19,7 +19,8 @@
 //     bypass the registers): one commit group per item, wait on the oldest,
 //     so two items are in flight while one is consumed;
 //   X': the CTA copies its X' chunk (all tokens, zero rows >= T) into shared
-//     memory;
+//     memory, one warp per token row; the decode rotation kernel writes X'
+//     already in the lane-major order the B fragments read;
 //   math: each 32-bit int4 word is dequantised in registers (LOP3 into the
 //     1024 + q bit pattern, exact fp16 subtraction of 1024 + z, one rounded
 //     fp16 multiply: w_hat = fp16((q - z) s)) straight into an m16n8k16 A

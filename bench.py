@@ -276,11 +276,12 @@ def bench_rotate(args, torch, B, local):
         g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
     per = e0.elapsed_time(e1) / 1e3 / (args.steps * len(xs))
     del g
     nbytes = 4 * T * n_in + K * (n_in // GROUP) * P * 10 + 4 * n_in
@@ -289,7 +290,7 @@ def bench_rotate(args, torch, B, local):
                       "us_per_call": per * 1e6, "GB/s": nbytes / per / 1e9,
                       "roofline": {"bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm_peak,
                                    "frac": nbytes / per / 1e9 / hbm_peak, "peak_source": kind},
-                      "copies": copies}), flush=True)
+                      "copies": copies, "clocks": clk.summary()}), flush=True)
     return 0
 
 

@@ -152,7 +152,8 @@ def decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_byte
         "config": config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
-                     "traffic": GEMV_TRAFFIC_PER_LAUNCH_T16 if args.tokens == 16 else None,
+                     "traffic": (GEMV_TRAFFIC_PER_LAUNCH_T16
+                                 if args.tokens == 16 and args.model == "llama3-8b" else None),
                      "kernel": "gemv_kernel (int4 decode)",
                      "us_per_launch": 1e6 * kern_s / (args.steps * n_calls),
                      "peak_source": f"{peak_kind} hbm_gbs"},

@@ -62,3 +62,26 @@ def test_single_process_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(None, [3, 1.5]) == [3.0, 1.5]
+
+
+def test_decode_line_carries_every_contract_key():
+    sys.path.insert(0, ROOT)
+    import bench
+    args = types.SimpleNamespace(steps=10, warmup=3, tokens=16, layers=4, gpus=1, model="llama3-8b")
+    line = bench.decode_line(args, 1, 2.0, 3.0, 1.0, step_bytes=1e9, gemv_bytes=5e8, n_calls=16,
+                             hbm_peak=6454.9, peak_kind="measured", h2d=1, d2h=2, per_proj={},
+                             n_launch=320, clocks={"sm_mhz": 1965.0})
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in line, k
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in line["roofline"], k
+    for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert k in line["e2e"], k
+    assert line["roofline"]["traffic"] == bench.GEMV_TRAFFIC_PER_LAUNCH_T16
+    assert line["e2e"]["value"] == pytest.approx(1e9 * 10 / 3.0 / 1e9)
+    json.dumps(line)
+    # the measured traffic belongs to one workload: no figure for another one
+    other = types.SimpleNamespace(**{**vars(args), "model": "qwen3-4b"})
+    assert bench.decode_line(other, 1, 2.0, 3.0, 1.0, 1e9, 5e8, 16, 6454.9, "measured", 1, 2, {}, 320,
+                             {})["roofline"]["traffic"] is None

@@ -132,8 +132,11 @@ paro_status paro_linear_workspace_size(int64_t tokens, int64_t in_features, int6
  *   qweight_dev, scales_dev, zeros_dev   from paro_pack_weights
  *   Y_dev         fp16 [tokens][out_features]
  *   workspace_dev at least paro_linear_workspace_size bytes of scratch (no
- *                 initialisation needed); it receives X T^-1 in fp16. Calls
- *                 that share a workspace must not overlap on the GPU.
+ *                 initialisation needed); it receives X T^-1 in fp16, in an
+ *                 internal order (for tokens <= 16 the channels of each
+ *                 64-channel block are permuted for the decode kernel), so
+ *                 its contents are not an output: use paro_rotate for X T^-1.
+ *                 Calls that share a workspace must not overlap on the GPU.
  * The rotation kernel writes X T^-1 into the workspace; the contraction runs
  * as a programmatic dependent launch of it (its weight loads start before the
  * rotation has finished). tokens <= 16: the int4 decode kernel (warp MMAs fed

@@ -91,13 +91,17 @@ paro_status paro_pack_size(int64_t in_features, int64_t out_features,
  * paro_linear (the int4 layout of the weight stream; one 16x16 tile is one
  * 32-bit word per lane of a warp, nibbles ordered for a two-instruction
  * int4->fp16 conversion).
- *   q_dev      uint8  [out][in], values 0..15
- *   s_dev      fp16   [out][in/128], the stored scales
- *   z_dev      uint8  [out][in/128], values 0..15
+ *   q          uint8  [out][in], values 0..15
+ *   s          fp16   [out][in/128], the stored scales
+ *   z          uint8  [out][in/128], values 0..15
+ *   q, s, z may be device memory (pinned host memory also works): the call
+ *   then enqueues on `stream` and returns. If any of them is plain host
+ *   memory, the three are staged through one temporary device allocation
+ *   and the call is synchronous (an offline step).
  *   qweight_dev, scales_dev, zeros_dev: outputs sized by paro_pack_size.
  * Paper: W4G128 (paper notes, main-experiment table heading); s and z are the
  * quantisation parameters named in the notes' training-strategy section. */
-paro_status paro_pack_weights(const uint8_t* q_dev, const uint16_t* s_dev, const uint8_t* z_dev,
+paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t* z,
                               int64_t in_features, int64_t out_features,
                               void* qweight_dev, void* scales_dev, void* zeros_dev,
                               paro_stream stream);
@@ -178,6 +182,27 @@ paro_status paro_linear_noalloc(const paro_rot* rot, const void* X_dev,
                                 const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
                                 void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,
                                 paro_stream stream);
+
+/* One-shot form of paro_rotate with the rotation given as the pages state
+ * it, X T^-1 from (pairs, theta, alpha, K, group) (CSDN article, section 2.1,
+ * the activation side; paper notes, "key design", T = (prod R) diag(alpha)).
+ * It runs paro_rot_create, paro_rotate and paro_rot_destroy in turn:
+ * allocating and synchronous, for one-off use; repeated calls should keep a
+ * handle. Arguments as in those calls (pairs/theta/alpha on the host, X and
+ * Xr fp16 [tokens][in_features] on the device). */
+paro_status paro_rotate_once(const void* X_dev, void* Xr_dev, int64_t tokens, int64_t in_features,
+                             const int16_t* pairs_host, const float* theta_host, const float* alpha_host,
+                             int K, int group, int pairs_per_group, paro_stream stream);
+
+/* One-shot form of paro_linear, Y = (X T^-1) w_hat^T from (X, pairs, theta,
+ * alpha, qweight, scales, zeros) (CSDN article, section 2.1, without the
+ * bias): paro_rot_create (group 128), a workspace from cudaMalloc,
+ * paro_linear, then everything is released; synchronous. Arguments as in
+ * paro_rot_create and paro_linear. */
+paro_status paro_linear_once(const void* X_dev, const int16_t* pairs_host, const float* theta_host,
+                             const float* alpha_host, const void* qweight_dev, const void* scales_dev,
+                             const void* zeros_dev, void* Y_dev, int64_t tokens, int64_t in_features,
+                             int64_t out_features, int K, int pairs_per_group, paro_stream stream);
 
 /* Fault word of the current device: 0, or the code of a bounded wait inside a
  * tensor-core kernel that ran out (about 2 s) because a pipeline stage never

@@ -36,6 +36,8 @@ _SIGS = {
     "paro_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
     "paro_linear_bias": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
     "paro_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
+    "paro_rotate_once": [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _int, _int, _int, _vp],
+    "paro_linear_once": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp],
     "paro_fault_status": [ctypes.POINTER(_int), _int],
     "paro_last_error": [],
 }
@@ -148,18 +150,26 @@ def paro_pack_size(in_features: int, out_features: int):
     return q.value, s.value, z.value
 
 
-def paro_pack_weights(q: torch.Tensor, s: torch.Tensor, z: torch.Tensor, stream=None):
-    """Logical (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]) on the
-    device -> device format (qweight, scales, zeros) as uint8 tensors."""
+def _any(t, dtype, name) -> int:
+    """Data pointer of a contiguous tensor on the device or on the host."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {dtype} tensor")
+    return t.data_ptr()
+
+
+def paro_pack_weights(q: torch.Tensor, s: torch.Tensor, z: torch.Tensor, stream=None, device=None):
+    """Logical (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]), on the
+    device or on the host -> device format (qweight, scales, zeros) as uint8
+    tensors on `device` (default: q's device, else the current one)."""
     out_f, in_f = q.shape
     qb, sb, zb = paro_pack_size(in_f, out_f)
-    dev = q.device
+    dev = device or (q.device if q.is_cuda else torch.device("cuda", torch.cuda.current_device()))
     qw = torch.empty(qb, dtype=torch.uint8, device=dev)
     sp = torch.empty(sb, dtype=torch.uint8, device=dev)
     zp = torch.empty(zb, dtype=torch.uint8, device=dev)
     _check("paro_pack_weights", lib().paro_pack_weights(
-        _dev(q, torch.uint8, "q"), _dev(s, torch.float16, "s"), _dev(z, torch.uint8, "z"), in_f, out_f,
-        qw.data_ptr(), sp.data_ptr(), zp.data_ptr(), _stream(stream)))
+        _any(q, torch.uint8, "q"), _any(s, torch.float16, "s"), _any(z, torch.uint8, "z"), in_f, out_f,
+        qw.data_ptr(), sp.data_ptr(), zp.data_ptr(), _stream(stream, qw.device)))
     return qw, sp, zp
 
 
@@ -228,6 +238,40 @@ def paro_linear_bias(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, bias:
         rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
         _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"), b,
         _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
+        _stream(stream, X.device)))
+    return Y
+
+
+def paro_rotate_once(X: torch.Tensor, pairs, theta, alpha, group: int = 128, stream=None) -> torch.Tensor:
+    """X T^-1 from (pairs, theta, alpha) without a handle (allocating, synchronous)."""
+    pairs = np.ascontiguousarray(pairs, dtype=np.int16)
+    theta = np.ascontiguousarray(theta, dtype=np.float32)
+    alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+    K = int(pairs.shape[0])
+    P = int(pairs.shape[2]) if K else 0
+    Xr = torch.empty_like(X)
+    T, in_f = X.shape
+    _check("paro_rotate_once", lib().paro_rotate_once(
+        _dev(X, torch.float16, "X"), _dev(Xr, torch.float16, "Xr"), T, in_f, pairs.ctypes.data if K else None,
+        theta.ctypes.data if K else None, alpha.ctypes.data, K, group, P, _stream(stream, X.device)))
+    return Xr
+
+
+def paro_linear_once(X: torch.Tensor, pairs, theta, alpha, qw, sp, zp, out_features: int,
+                     stream=None) -> torch.Tensor:
+    """Y = (X T^-1) w_hat^T from (pairs, theta, alpha) without a handle
+    (allocating, synchronous)."""
+    pairs = np.ascontiguousarray(pairs, dtype=np.int16)
+    theta = np.ascontiguousarray(theta, dtype=np.float32)
+    alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+    K = int(pairs.shape[0])
+    P = int(pairs.shape[2]) if K else 0
+    T, in_f = X.shape
+    Y = torch.empty((T, out_features), dtype=torch.float16, device=X.device)
+    _check("paro_linear_once", lib().paro_linear_once(
+        _dev(X, torch.float16, "X"), pairs.ctypes.data if K else None, theta.ctypes.data if K else None,
+        alpha.ctypes.data, _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"),
+        _dev(zp, torch.uint8, "zeros"), _dev(Y, torch.float16, "Y"), T, in_f, out_features, K, P,
         _stream(stream, X.device)))
     return Y
 

@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -270,16 +271,23 @@ template <int BN, int STAGES, int DQG, int NACC>
 cudaError_t launch_cfg(const CUtensorMap* tm, const GemmArgs& a, int mt, int nt, cudaStream_t s) {
     constexpr size_t smem = STAGES * (BN * 128 + kWStage + kSStage + kZStage) + (3 * STAGES + 2) * 8 +
                             16 * (128 + 4) * 4 + 1024;
-    static bool configured[64] = {};
+    // kernel attributes, set once per device (double-checked under a lock)
+    static std::atomic<bool> configured[64] = {};
+    static std::mutex mu;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_w4_kernel<BN, STAGES, DQG, NACC>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gemm_w4_kernel<BN, STAGES, DQG, NACC>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!configured[dev].load(std::memory_order_relaxed)) {
+            cudaError_t e = cudaFuncSetAttribute(gemm_w4_kernel<BN, STAGES, DQG, NACC>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gemm_w4_kernel<BN, STAGES, DQG, NACC>,
+                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            configured[dev].store(true, std::memory_order_release);
+        }
     }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(mt, nt, a.nsplit);

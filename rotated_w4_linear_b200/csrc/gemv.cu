@@ -34,6 +34,7 @@
 // The k order inside each 16x16 tile follows the packed layout: the MMA's
 // logical k slot 2q+e holds channel 4q+e and slot 2q+8+e channel 4q+2+e.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <map>
 #include <mutex>
@@ -525,16 +526,21 @@ GemvPlan cached_plan(int dev, int64_t in, int64_t out, int T, int K) {
 }
 
 template <int NT>
-cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, cudaStream_t s) {
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
+cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, int dev, cudaStream_t s) {
+    // kernel attributes, set once per device (double-checked under a lock)
+    static std::atomic<bool> configured[64] = {};
+    static std::mutex mu;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!configured[dev].load(std::memory_order_relaxed)) {
+            cudaError_t e =
+                cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            configured[dev].store(true, std::memory_order_release);
+        }
     }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(p.nsplit, p.rowtiles, 1);
@@ -590,7 +596,7 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.bias = static_cast<const __half*>(bias);
     a.Y = static_cast<__half*>(Y);
     a.xlm = rot ? 1 : 0;
-    cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, s) : launch_gemv_t<1>(a, p, s);
+    cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, dev, s) : launch_gemv_t<1>(a, p, dev, s);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -612,19 +618,29 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;   // 1 MiB: e.g. 16 tokens x 32768 channels
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch, looked up once per device (in host
-// code the array's name is only a host-side stand-in, not a device address).
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (in host code the array's name is only a host-side stand-in,
+// not a device address). The lookup is guarded by a lock, so threads making
+// their first call on one device at once do not race. The address is kept for
+// the life of the process: a context reset (cudaDeviceReset) invalidates it,
+// and calls after such a reset are not supported.
 cudaError_t noalloc_scratch(void** ptr) {
     static void* addr[64] = {};
-    static bool ready[64] = {};
+    static std::atomic<bool> ready[64] = {};
+    static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!ready[dev]) {
-        e = cudaGetSymbolAddress(&addr[dev], g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        ready[dev] = true;
+    if (!ready[dev].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!ready[dev].load(std::memory_order_relaxed)) {
+            void* a = nullptr;
+            e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+            if (e != cudaSuccess) return e;
+            addr[dev] = a;
+            ready[dev].store(true, std::memory_order_release);
+        }
     }
     *ptr = addr[dev];
     return cudaSuccess;

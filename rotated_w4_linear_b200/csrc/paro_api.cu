@@ -60,6 +60,17 @@ paro_status check_shape(int64_t in, int64_t out) {
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+// Plain host memory (not allocated or registered with CUDA) that a kernel
+// cannot read.
+bool is_unregistered_host(const void* p) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return true;
+    }
+    return a.type == cudaMemoryTypeUnregistered;
+}
+
 }  // namespace
 
 extern "C" {
@@ -330,8 +341,29 @@ paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t
     if (st != PARO_OK) return st;
     if (!q || !s || !z || !qw || !sp || !zp) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(qw) || !aligned16(sp) || !aligned16(zp)) return fail(PARO_ERR_ARG, "outputs must be 16-byte aligned");
-    cudaError_t e = paro::launch_pack(q, s, z, in, out, qw, sp, zp, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "pack launch");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (!is_unregistered_host(q) && !is_unregistered_host(s) && !is_unregistered_host(z)) {
+        cudaError_t e = paro::launch_pack(q, s, z, in, out, qw, sp, zp, cs);
+        return e == cudaSuccess ? PARO_OK : cuda_fail(e, "pack launch");
+    }
+    // host inputs: stage the logical tensors in one temporary device buffer
+    // (offline step; synchronous on `stream`)
+    const size_t G = (size_t)(in / 128);
+    const size_t nq = (size_t)in * (size_t)out, ns = (size_t)out * G * 2, nz = (size_t)out * G;
+    const size_t oq = 0, os_ = round256(nq), oz = os_ + round256(ns), total = oz + round256(nz);
+    char* tmp = nullptr;
+    cudaError_t e = cudaMalloc(&tmp, total);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(staging of host q/s/z)");
+    e = cudaMemcpyAsync(tmp + oq, q, nq, cudaMemcpyDefault, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(tmp + os_, s, ns, cudaMemcpyDefault, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(tmp + oz, z, nz, cudaMemcpyDefault, cs);
+    if (e == cudaSuccess)
+        e = paro::launch_pack(reinterpret_cast<const uint8_t*>(tmp + oq), reinterpret_cast<const uint16_t*>(tmp + os_),
+                              reinterpret_cast<const uint8_t*>(tmp + oz), in, out, qw, sp, zp, cs);
+    const cudaError_t e2 = cudaStreamSynchronize(cs);
+    cudaFree(tmp);
+    if (e != cudaSuccess) return cuda_fail(e, "pack from host memory");
+    return e2 == cudaSuccess ? PARO_OK : cuda_fail(e2, "pack from host memory (synchronize)");
 }
 
 paro_status paro_dequant(const void* qw, const void* sp, const void* zp, int64_t in, int64_t out, void* W,
@@ -362,7 +394,7 @@ paro_status paro_linear_workspace_size(int64_t T, int64_t in, int64_t out, size_
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
     if (T < 0 || !bytes) return fail(PARO_ERR_ARG, "bad tokens or null bytes");
-    *bytes = round256((size_t)(T < 16 ? 16 : T) * in * 2);   // X T^-1 (fp16)
+    *bytes = round256((size_t)T * in * 2);   // X T^-1 (fp16), one row per token
     return PARO_OK;
 }
 
@@ -405,6 +437,44 @@ paro_status paro_linear_bias(const paro_rot* r, const void* X, const void* qw, c
 paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp, void* Y,
                         int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes, paro_stream stream) {
     return paro_linear_bias(r, X, qw, sp, zp, nullptr, Y, T, in, out, ws, ws_bytes, stream);
+}
+
+// One-shot forms: prepare the rotation, run the call, release everything
+// (allocating and synchronous; the handle calls above are the hot path).
+paro_status paro_rotate_once(const void* X, void* Xr, int64_t T, int64_t in, const int16_t* pairs,
+                             const float* theta, const float* alpha, int K, int group, int pairs_per_group,
+                             paro_stream stream) {
+    paro_rot* r = nullptr;
+    paro_status st = paro_rot_create(&r, in, group, K, pairs_per_group, pairs, theta, alpha);
+    if (st != PARO_OK) return st;
+    st = paro_rotate(r, X, Xr, T, stream);
+    if (st == PARO_OK) {
+        const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) st = cuda_fail(e, "synchronize");
+    }
+    const paro_status st2 = paro_rot_destroy(r);
+    return st != PARO_OK ? st : st2;
+}
+
+paro_status paro_linear_once(const void* X, const int16_t* pairs, const float* theta, const float* alpha,
+                             const void* qweight, const void* scales, const void* zeros, void* Y, int64_t T,
+                             int64_t in, int64_t out, int K, int pairs_per_group, paro_stream stream) {
+    paro_rot* r = nullptr;
+    paro_status st = paro_rot_create(&r, in, 128, K, pairs_per_group, pairs, theta, alpha);
+    if (st != PARO_OK) return st;
+    size_t ws_bytes = 0;
+    void* ws = nullptr;
+    st = paro_linear_workspace_size(T, in, out, &ws_bytes);
+    if (st == PARO_OK && ws_bytes > 0) {
+        const cudaError_t e = cudaMalloc(&ws, ws_bytes);
+        if (e != cudaSuccess) st = cuda_fail(e, "cudaMalloc(workspace)");
+    }
+    if (st == PARO_OK) st = paro_linear(r, X, qweight, scales, zeros, Y, T, in, out, ws ? ws : Y, ws_bytes, stream);
+    const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (st == PARO_OK && e != cudaSuccess) st = cuda_fail(e, "synchronize");
+    if (ws) cudaFree(ws);
+    const paro_status st2 = paro_rot_destroy(r);
+    return st != PARO_OK ? st : st2;
 }
 
 }  // extern "C"

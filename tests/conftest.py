@@ -8,8 +8,22 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+# Parity figures recorded by the GPU tests (test, quantity, value, bound),
+# printed after the run so the literal errors are visible beside the bars.
+PARITY = []
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_terminal_summary(terminalreporter):
+    if not PARITY:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "parity with the fp64 oracle (literal figures)")
+    for test, what, value, bound in PARITY:
+        tr.write_line(f"{test:<70} {what:<34} {value:.3e}  (bar {bound})")
 
 
 @pytest.fixture(scope="session")

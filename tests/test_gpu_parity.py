@@ -1,23 +1,31 @@
 """Parity of the CUDA path (through the C ABI) with the CPU fp64 oracle.
 
-Tolerances (stated by the task for this layer, with the readings of the
-open points):
+Tolerances (stated for this layer, with the readings of the open points):
   * int4 unpack/dequant: bit-exact fp16;
   * offline quantiser: bit-exact q, s, z;
   * rotated activations: per-element relative error <= 1e-3 against fp64,
-    the denominator floored at 1% of the element's group maximum;
+    the denominator floored at 1% of the element's group maximum (the
+    literal, unfloored maximum is recorded beside it);
   * layer output: ||Y - Y_ref|| / ||Y_ref|| <= 2e-3, and per element
-    |Y - Y_ref| <= max(1e-2, |Y_x16 - Y_ref| + ulp16(Y_ref) + 2e-3), where
-    Y_x16 is the exact contraction of the fp16-rounded X' (before the output
-    is rounded): an element may exceed 1e-2 only by its own fp16 format
-    floor (the X' rounding plus rounding to either fp16 neighbour).
+    |Y - Y_ref| <= max(1e-2, f + 2e-3), where f = |Y_x16 - Y_ref| +
+    spacing16/2 is that element's error in the ideal fp16 pipeline (X'
+    rounded to fp16, exact contraction, Y rounded to nearest fp16: Y_x16 is
+    its value before the output rounding, spacing16 the fp16 spacing at the
+    larger of |Y| and |Y_ref|) and 2e-3 the budget for fp32 accumulation and
+    for X' elements that round to the other fp16 neighbour. An element may
+    pass above 1e-2 only where the format itself forces it, and a result
+    rounded to the wrong fp16 neighbour passes only within that budget of a
+    rounding midpoint (tests/test_parity_bounds.py). The literal max |Y - Y_ref| and the pipeline's own maximum
+    (the format floor) are recorded for every call.
 """
+
 import numpy as np
 import pytest
 import torch
 
 import synth
 from oracle import paro_oracle as O
+from parity import check_linear, check_rotation
 
 pytestmark = pytest.mark.gpu
 
@@ -34,35 +42,6 @@ def dev(a):
 
 def host(t):
     return t.detach().cpu().numpy()
-
-
-ROT_TOL = 1e-3
-REL_TOL = 2e-3
-ABS_TOL = 1e-2
-
-
-def check_rotation(got16, x, pairs, theta, alpha):
-    ref = O.rotate_activations(x, pairs, theta, alpha)
-    fl, lit = O.rotation_rel_error(got16.astype(np.float64), ref)
-    assert fl <= ROT_TOL, (fl, lit)
-    return fl
-
-
-def check_linear(y16, x, pairs, theta, alpha, q, s, z, bias=None):
-    if pairs is None:                       # unrotated layer: theta = 0, alpha = 1
-        pairs, theta, alpha = synth.rotation_params(x.shape[1], 1, 0)
-        theta = np.zeros_like(theta)
-        alpha = np.ones_like(alpha)
-    ref = O.linear(x, pairs, theta, alpha, q, s, z, bias=bias)
-    x16 = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, round_output=False, bias=bias)
-    y = y16.astype(np.float64)
-    rel, mx = O.output_errors(y, ref)
-    ulp = np.abs(np.spacing(np.abs(ref).astype(np.float16))).astype(np.float64)
-    bound = np.maximum(ABS_TOL, np.abs(x16 - ref) + ulp + 2e-3)
-    worst = float(np.max(np.abs(y - ref) - bound)) if y.size else 0.0
-    assert rel <= REL_TOL, (rel, mx)
-    assert worst <= 0.0, (rel, mx, worst)
-    return rel, mx
 
 
 # ---------------------------------------------------------------- rotation
@@ -294,35 +273,55 @@ def test_linear_decode_qwen3_shapes_sampled(B, T, in_f, out_f):
     check_linear(y[:, rows], x, pairs, theta, alpha, q[rows], s[rows], z[rows])
 
 
-@pytest.mark.parametrize("in_f,out_f", [(2560, 6144), (9728, 2560), (5120, 34816), (17408, 5120)])
+def _prefill_sampled(B, T, in_f, out_f, seed, n_tok=16, n_rows=128):
+    """One full-size prefill call; the oracle checks n_tok sampled tokens
+    (first and last included) over n_rows sampled output rows (first and
+    last included)."""
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+    q, s, z = synth.w4_codes(out_f, in_f, seed)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    y = B.paro_linear(rot, dev(x), qw, sp, zp, out_f)
+    rng = np.random.default_rng(seed)
+    toks = rng.choice(T, n_tok, replace=False)
+    toks[0], toks[-1] = 0, T - 1
+    rows = rng.choice(out_f, n_rows, replace=False)
+    rows[0], rows[-1] = 0, out_f - 1
+    ys = host(y[torch.from_numpy(toks).cuda()][:, torch.from_numpy(rows).cuda()])
+    del y
+    check_linear(ys, x[toks], pairs, theta, alpha, q[rows], s[rows], z[rows])
+    assert B.paro_fault_status() == 0
+
+
+@pytest.mark.parametrize("in_f,out_f", QWEN3)
 def test_linear_prefill_qwen3_shapes_sampled(B, in_f, out_f):
-    T = 4096
-    seed = synth.layer_seed(4, in_f + out_f)
-    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
-    q, s, z = synth.w4_codes(out_f, in_f, seed)
-    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
-    x = synth.activations(T, in_f, seed)
-    rot = B.paro_rot_create(pairs, theta, alpha)
-    y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
-    rng = np.random.default_rng(seed)
-    toks = rng.choice(T, 16, replace=False)
-    toks[0], toks[-1] = 0, T - 1
-    rows = rng.choice(out_f, 128, replace=False)
-    check_linear(y[np.ix_(toks, rows)], x[toks], pairs, theta, alpha, q[rows], s[rows], z[rows])
+    _prefill_sampled(B, 4096, in_f, out_f, synth.layer_seed(4, in_f + out_f))
 
 
-@pytest.mark.parametrize("in_f,out_f", [(4096, 4096), (14336, 4096)])
-def test_linear_prefill_full_size_sampled(B, in_f, out_f):
-    T = 2048
-    seed = synth.layer_seed(3, in_f + out_f)
-    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
-    q, s, z = synth.w4_codes(out_f, in_f, seed)
-    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+@pytest.mark.parametrize("T", [2048, 8192])
+@pytest.mark.parametrize("in_f,out_f", LLAMA)
+def test_linear_prefill_full_size_sampled(B, T, in_f, out_f):
+    _prefill_sampled(B, T, in_f, out_f, synth.layer_seed(3, in_f + out_f + T), n_tok=24, n_rows=256)
+
+
+@pytest.mark.parametrize("T", [5, 300])
+def test_oneshot_calls_and_host_packing(B, T):
+    """paro_rotate_once / paro_linear_once (the rotation given as pairs,
+    theta, alpha) give the handle calls' bits; packing from host tensors
+    gives the device packing's bytes."""
+    in_f, out_f = 512, 96
+    seed = synth.layer_seed(7, T)
+    (pairs, theta, alpha, q, s, z), (qw, sp, zp) = _layer(B, in_f, out_f, 8, 64, seed)
+    qh, sh, zh = (B.paro_pack_weights(torch.from_numpy(q), torch.from_numpy(s), torch.from_numpy(z)))
+    for a, b in ((qw, qh), (sp, sh), (zp, zh)):
+        assert torch.equal(a, b)
     x = synth.activations(T, in_f, seed)
     rot = B.paro_rot_create(pairs, theta, alpha)
+    xr = host(B.paro_rotate(rot, dev(x)))
+    xr1 = host(B.paro_rotate_once(dev(x), pairs, theta, alpha))
+    assert np.array_equal(xr.view(np.uint16), xr1.view(np.uint16))
     y = host(B.paro_linear(rot, dev(x), qw, sp, zp, out_f))
-    rng = np.random.default_rng(seed)
-    toks = rng.choice(T, 24, replace=False)
-    toks[0], toks[-1] = 0, T - 1
-    rows = rng.choice(out_f, 256, replace=False)
-    check_linear(y[np.ix_(toks, rows)], x[toks], pairs, theta, alpha, q[rows], s[rows], z[rows])
+    y1 = host(B.paro_linear_once(dev(x), pairs, theta, alpha, qh, sh, zh, out_f))
+    assert np.array_equal(y.view(np.uint16), y1.view(np.uint16))
+    check_linear(y1, x, pairs, theta, alpha, q, s, z)

@@ -270,3 +270,42 @@ def test_bias_is_added_once_per_output_column():
     yb = O.linear(x, pairs, theta, alpha, q, s, z, bias=b)
     bb = np.broadcast_to(b.astype(np.float64), (T, out_f))
     assert np.all(np.abs((yb - ya) - bb) <= 1e-12 * (np.abs(ya) + np.abs(bb)))
+
+
+# ---- the ideal fp16 pipeline (format floor of the output tolerance) ------------
+def _fp16_pipeline_layer():
+    """The tiny layer of tests/golden/fp16_pipeline.txt: one group, one layer
+    with pair (0, 1) at theta = 0, alpha = 3, two output rows."""
+    pairs = np.zeros((1, 1, 1, 2), np.int16)
+    pairs[0, 0, 0] = (0, 1)
+    theta = np.zeros((1, 1, 1), np.float32)
+    alpha = np.full(128, 3.0, np.float32)
+    q = np.zeros((2, 128), np.uint8)
+    q[0, :2] = 3
+    q[1, :] = 1
+    q[1, 0], q[1, 1] = 2, 0
+    z = np.array([[0], [1]], np.uint8)
+    s = np.ones((2, 1), np.float16)
+    rows = {r[0]: [float(v) for v in r[1:]] for r in _rows("fp16_pipeline.txt")}
+    x = np.zeros((2, 128), np.float16)
+    x[0, :2], x[1, :2] = rows["x0"], rows["x1"]
+    return (x, pairs, theta, alpha, q, s, z), rows
+
+
+def test_fp16_pipeline_golden():
+    """X' rounded to fp16, exact contraction, Y rounded to fp16 (or not), with
+    and without a bias: every value worked by hand, including three
+    round-half-to-even ties."""
+    layer, rows = _fp16_pipeline_layer()
+    b = np.array(rows["bias"], np.float16)
+    un = O.linear_fp16_pipeline(*layer, round_output=False)
+    rd = O.linear_fp16_pipeline(*layer, round_output=True)
+    assert un.dtype == np.float64 and rd.dtype == np.float16
+    assert un.reshape(-1).tolist() == rows["unrounded"]
+    assert rd.astype(np.float64).reshape(-1).tolist() == rows["rounded"]
+    unb = O.linear_fp16_pipeline(*layer, round_output=False, bias=b)
+    rdb = O.linear_fp16_pipeline(*layer, round_output=True, bias=b)
+    assert unb.reshape(-1).tolist() == rows["unrounded_bias"]
+    assert rdb.astype(np.float64).reshape(-1).tolist() == rows["rounded_bias"]
+    # the exact layer does not round X': the ties above do not arise there
+    assert np.allclose(O.linear(*layer).reshape(-1), rows["exact"], rtol=0, atol=1e-15)

@@ -204,11 +204,24 @@ paro_status paro_linear_once(const void* X_dev, const int16_t* pairs_host, const
                              const void* zeros_dev, void* Y_dev, int64_t tokens, int64_t in_features,
                              int64_t out_features, int K, int pairs_per_group, paro_stream stream);
 
-/* Fault word of the current device: 0, or the code of a bounded wait inside a
- * tensor-core kernel that ran out (about 2 s) because a pipeline stage never
- * arrived; the kernel then abandoned its tile instead of hanging, and its
- * output is not valid. Synchronous (copies one word); clear != 0 resets it. */
+/* Fault word of the current device: 0, or the code of a bounded wait inside
+ * a tensor-core kernel that ran out (about 2 s) because a pipeline stage
+ * never arrived: 1 TMA producer, 2 MMA issuer, 3 dequantisation, 4 epilogue,
+ * 5 a drain before exit, 6 the self-test below. The CTA that saw it raises an
+ * abort flag in its shared memory: every role stops issuing copies and
+ * MMAs, the copies and MMAs already issued are waited for (bounded), tensor
+ * memory is released and the CTA exits without storing its tile. The output
+ * of that call is not valid. Synchronous (copies one word); clear != 0
+ * resets it to 0. */
 paro_status paro_fault_status(int* code, int clear);
+
+/* Self-test of the failure detection (no counterpart in the paper): enqueue
+ * a one-thread kernel that waits, with a limit of limit_us microseconds
+ * (1..2000000), on an mbarrier at which nothing arrives, with no copy or MMA
+ * in flight. The wait runs out, records code 6 in the fault word and the
+ * kernel returns; the context stays usable. Read and clear the code with
+ * paro_fault_status. */
+paro_status paro_check_wait_timeout(uint32_t limit_us, paro_stream stream);
 
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* paro_last_error(void);

@@ -39,6 +39,7 @@ _SIGS = {
     "paro_rotate_once": [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _int, _int, _int, _vp],
     "paro_linear_once": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp],
     "paro_fault_status": [ctypes.POINTER(_int), _int],
+    "paro_check_wait_timeout": [ctypes.c_uint32, _vp],
     "paro_last_error": [],
 }
 
@@ -142,6 +143,11 @@ def paro_fault_status(clear: bool = False) -> int:
     c = _int()
     _check("paro_fault_status", lib().paro_fault_status(ctypes.byref(c), 1 if clear else 0))
     return c.value
+
+
+def paro_check_wait_timeout(limit_us: int = 1000, stream=None) -> None:
+    """Enqueue the self-test kernel whose bounded wait runs out (code 6)."""
+    _check("paro_check_wait_timeout", lib().paro_check_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def paro_pack_size(in_features: int, out_features: int):

@@ -92,6 +92,8 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     unsigned char* sZ = sS + STAGES * kSStage;          // per stage: zeros of the group pair, 8 row blocks x 16 B
     uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + STAGES * kZStage);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
+    // raised by a wait that ran out: every role stops issuing work (tslot[1])
+    volatile uint32_t* abort = tslot + 1;
     float* red = reinterpret_cast<float*>(bars + 3 * STAGES + 2);   // split-k partial tile (BN == 16)
     const uint32_t full0 = smem_addr(bars), afull0 = full0 + 8 * STAGES, free0 = afull0 + 8 * STAGES;
     const uint32_t done = free0 + 8 * STAGES;
@@ -113,6 +115,7 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             mbar_init(free0 + 8 * s, 1);
         }
         mbar_init(done, 1);
+        *abort = 0u;
         mbar_fence_init();
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_w);
@@ -130,23 +133,37 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
     if (warp == 0) {
         if (lane == 0) {
+            // issued[s]: stage s's loads issued so far (the last one's phase
+            // is issued[s] - 1); they must all have landed before the CTA exits
+            int issued[STAGES];
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s) issued[s] = 0;
             for (int i = 0; i < nk; ++i) {
                 const int s = i % STAGES, u = i / STAGES;
-                if (u > 0) mbar_wait(free0 + 8 * s, (u - 1) & 1, kFaultTmaWait);
+                if (u > 0 && !mbar_wait(free0 + 8 * s, (u - 1) & 1, kFaultTmaWait, abort)) break;
+                if (*abort) break;
                 const int kb = kblock(i), gi = kb >> 1;
                 mbar_arrive_expect_tx(full0 + 8 * s, kBStage + kWStage + kSStage + kZStage);
                 tma_load_2d(smem_addr(sB + s * kBStage), &tm_x, kb * 64, n0, full0 + 8 * s);
                 tma_load_2d(smem_addr(sW + s * kWStage), &tm_w, kb * 128, rb0, full0 + 8 * s);
                 tma_load_2d(smem_addr(sS + s * kSStage), &tm_s, gi * 8, rb0, full0 + 8 * s);
                 tma_load_2d(smem_addr(sZ + s * kZStage), &tm_z, (gi & ~1) * 8, rb0, full0 + 8 * s);
+#pragma unroll
+                for (int t = 0; t < STAGES; ++t)
+                    if (t == s) issued[t] = u + 1;
+            }
+            if (*abort) {   // drain: wait (bounded, not cut short) for every issued load to land
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s] > 0) mbar_wait(full0 + 8 * s, (issued[s] - 1) & 1, kFaultDrainWait, nullptr);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             for (int i = 0; i < nk; ++i) {
                 const int s = i % STAGES, u = i / STAGES;
-                mbar_wait(afull0 + 8 * s, u & 1, kFaultMmaWait);
-                mbar_wait(full0 + 8 * s, u & 1, kFaultMmaWait);
+                if (!mbar_wait(afull0 + 8 * s, u & 1, kFaultMmaWait, abort)) break;
+                if (!mbar_wait(full0 + 8 * s, u & 1, kFaultMmaWait, abort)) break;
                 tc_fence_after();
                 const uint64_t bdesc = umma_desc_sw128_kmajor(smem_addr(sB + s * kBStage));
 #pragma unroll
@@ -157,6 +174,8 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
                 umma_commit(free0 + 8 * s);
             }
+            // always: `done` arrives once every MMA issued above has completed
+            // (also after an abort, so tensor memory is released only then)
             umma_commit(done);
         }
     } else {
@@ -167,7 +186,10 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         for (int i = dg; i < nk; i += DQG) {
             const int s = i % STAGES, u = i / STAGES;
             const int gi = kblock(i) >> 1;
-            mbar_wait(full0 + 8 * s, u & 1, kFaultDequantWait);
+            // the tensor-memory stores below are warp-collective: the whole
+            // warp goes on only if every lane saw the stage arrive
+            if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8 * s, u & 1, kFaultDequantWait, abort) && !*abort))
+                break;
             const uint32_t wbase = smem_addr(sW + s * kWStage);
             const uint32_t sbase = smem_addr(sS + s * kSStage), zbase = smem_addr(sZ + s * kZStage);
 #pragma unroll
@@ -190,8 +212,8 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         }
 
         // ---- epilogue (group 0): one accumulator row per thread
-        if (dg == 0) {
-            mbar_wait(done, 0, kFaultEpilogueWait);
+        // (skipped after an abort: the tile is not valid, and the fault word says so)
+        if (dg == 0 && __all_sync(0xffffffffu, mbar_wait(done, 0, kFaultEpilogueWait, abort) && !*abort)) {
             tc_fence_after();
             const int rloc = 32 * qw + lane;
             const int row = rb0 * 16 + rloc;
@@ -244,6 +266,10 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         __syncthreads();
     }
     if (warp == 1) {
+        // no MMA may still write tensor memory when it is released: `done`
+        // (committed after the last MMA this CTA issued) must have arrived;
+        // this wait is not cut short by the abort flag
+        mbar_wait(done, 0, kFaultDrainWait, nullptr);
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }
@@ -368,6 +394,26 @@ cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const v
     else if (BN == 128) e = launch_cfg<128, 4, 1, 1>(tm, a, mt, nt, s);
     else e = launch_cfg<256, 4, 1, 1>(tm, a, mt, nt, s);
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// Self-test of the bounded waits: one thread waits on an mbarrier at which
+// nothing ever arrives (no copy or MMA is in flight). The wait runs out after
+// limit_ns, records kFaultSelfTest in the fault word and the kernel returns.
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        abort_flag = 0u;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, kFaultSelfTest, &abort_flag, limit_ns);
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s) {
+    wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns);
     return cudaGetLastError();
 }
 

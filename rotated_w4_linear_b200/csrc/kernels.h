@@ -49,6 +49,9 @@ cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw
 cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, const void* bias, void* Y,
                         int64_t T, int64_t in, int64_t out, cudaStream_t s);
 
+// A kernel whose bounded wait runs out on purpose after limit_ns (fault code 6).
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);
+
 // Fault code left by a bounded wait that ran out (0 = none); optionally cleared.
 cudaError_t read_fault(unsigned int* code, bool clear);
 

@@ -107,6 +107,15 @@ paro_status paro_fault_status(int* code, int clear) {
     return PARO_OK;
 }
 
+paro_status paro_check_wait_timeout(uint32_t limit_us, paro_stream stream) {
+    g_err[0] = 0;
+    if (limit_us < 1 || limit_us > 2000000) return fail(PARO_ERR_ARG, "limit_us=%u must be in 1..2000000", limit_us);
+    paro_status st = check_device();
+    if (st != PARO_OK) return st;
+    cudaError_t e = paro::launch_wait_selftest((uint64_t)limit_us * 1000ull, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "wait self-test launch");
+}
+
 paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P, const int16_t* pairs,
                             const float* theta, const float* alpha) {
     g_err[0] = 0;

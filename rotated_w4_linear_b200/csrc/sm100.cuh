@@ -1,8 +1,9 @@
 // Thin wrappers over the sm_100a instructions the tensor-core kernels use:
 // mbarriers, TMA tile loads, tcgen05 (TMEM allocation, MMA, commit, TMEM
 // loads/stores and their fences). Every wait is bounded: after a time limit
-// the waiting thread records a fault code in g_paro_fault and gives up, so
-// a logic error cannot hang the GPU.
+// the waiting thread records a fault code in g_paro_fault, raises the CTA's
+// abort flag and gives up, so a logic error cannot hang the GPU; a wait that
+// sees the abort flag raised by another thread of the CTA gives up at once.
 #pragma once
 
 #include <stdint.h>
@@ -14,7 +15,10 @@ namespace paro {
 static __device__ unsigned int g_paro_fault = 0;
 
 enum : unsigned int { kFaultTmaWait = 1, kFaultMmaWait = 2, kFaultDequantWait = 3, kFaultEpilogueWait = 4,
-                      kFaultDrainWait = 5 };
+                      kFaultDrainWait = 5, kFaultSelfTest = 6 };
+
+// Time limit of a pipeline wait: far above any stage of a correct kernel.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -44,15 +48,23 @@ __device__ __forceinline__ uint64_t global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for the phase with the given parity; give up after ~2 s (fault code).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int fault) {
+// Wait for the phase with the given parity. Returns false, without waiting
+// further, when `limit_ns` passes (the fault code is recorded and *abort is
+// raised) or when *abort is raised by another thread of the CTA (abort may
+// be null: a drain wait that must not be cut short by the flag).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int fault,
+                                          volatile uint32_t* abort, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0 && global_ns() - t0 > 2000000000ull) {
-            atomicCAS(&g_paro_fault, 0u, fault);
-            return false;
+        if ((it & 255u) == 0) {
+            if (abort && *abort) return false;
+            if (global_ns() - t0 > limit_ns) {
+                atomicCAS(&g_paro_fault, 0u, fault);
+                if (abort) *abort = 1u;
+                return false;
+            }
         }
     }
 }

@@ -64,6 +64,12 @@ def test_null_arguments_rejected_before_any_launch(L):
     assert L.paro_rot_destroy(None) == 0
 
 
+def test_wait_selftest_limit_checked_before_launch(L):
+    assert L.paro_check_wait_timeout(0, None) == 1
+    assert L.paro_check_wait_timeout(2000001, None) == 1
+    assert b"limit_us" in L.paro_last_error()
+
+
 def test_unsupported_group(L):
     h = ctypes.c_void_p()
     assert L.paro_rot_create(ctypes.byref(h), 256, 64, 8, 32, None, None, None) == 2

@@ -325,3 +325,22 @@ def test_oneshot_calls_and_host_packing(B, T):
     y1 = host(B.paro_linear_once(dev(x), pairs, theta, alpha, qh, sh, zh, out_f))
     assert np.array_equal(y.view(np.uint16), y1.view(np.uint16))
     check_linear(y1, x, pairs, theta, alpha, q, s, z)
+
+
+def test_bounded_wait_runs_out_and_the_context_survives(B):
+    """Failure detection without a GPU fault: a kernel waits, with a 1 ms
+    limit, on an mbarrier at which nothing arrives; the wait gives up, the
+    kernel returns, the fault word holds code 6 until cleared, and the next
+    layer call on the same context is correct."""
+    B.paro_fault_status(clear=True)
+    B.paro_check_wait_timeout(1000)
+    torch.cuda.synchronize()
+    assert B.paro_fault_status() == 6
+    assert B.paro_fault_status(clear=True) == 6
+    assert B.paro_fault_status() == 0
+    seed = synth.layer_seed(8, 1)
+    (pairs, theta, alpha, q, s, z), (qw, sp, zp) = _layer(B, 384, 48, 8, 64, seed)
+    x = synth.activations(40, 384, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    check_linear(host(B.paro_linear(rot, dev(x), qw, sp, zp, 48)), x, pairs, theta, alpha, q, s, z)
+    assert B.paro_fault_status() == 0

@@ -4,10 +4,12 @@ It serves callers that cannot allocate device memory: a serving engine that
 hands all device memory to its own pool at start-up, or code that must not
 call cudaMalloc while a CUDA graph is being captured. It runs the same
 kernels with the same plan as paro_linear, only with its X T^-1 scratch in a
-static device array, so its output must equal paro_linear's bit for bit, on
-two calls in a row (the array keeps the previous call's contents, here from a
-larger batch, which must not leak into the next). One call is also checked
-against the CPU fp64 oracle at the parity tolerances of the other tests.
+static device array. Its output must agree with paro_linear's within the
+parity tolerances the other tests use, on two calls in a row (the array keeps
+the previous call's contents, here from a larger batch, which must not leak
+into the next); both calls are also checked against the CPU fp64 oracle.
+(The decode kernel adds warp partial sums with shared-memory atomics, whose
+order varies from run to run, so two calls may differ in the last bit.)
 Collected last on purpose: if it fails, a run that stops at the first
 failure has already run every other test."""
 import numpy as np
@@ -16,7 +18,7 @@ import torch
 
 import synth
 from oracle import paro_oracle as O  # noqa: F401  (used through parity.check_linear)
-from parity import check_linear
+from parity import check_linear, output_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -41,10 +43,12 @@ def test_noalloc_matches_paro_linear_twice(cuda_lib):
                                    Y.data_ptr(), T, n_in, n_out, stream)
         assert st == 0, L.paro_last_error()
         torch.cuda.synchronize()
-        got = Y.cpu().numpy()
-        assert np.array_equal(got.view(np.uint16), ref.cpu().numpy().view(np.uint16)), call
-        if call == 1:
-            check_linear(got, x, pairs, theta, alpha, q, s, z)
+        got, want = Y.cpu().numpy(), ref.cpu().numpy()
+        a, b = got.astype(np.float64), want.astype(np.float64)
+        assert np.all(np.isfinite(a))
+        assert np.linalg.norm(a - b) <= 2e-3 * np.linalg.norm(b), call
+        assert np.all(np.abs(a - b) <= output_bound(a, b, b)), call
+        check_linear(got, x, pairs, theta, alpha, q, s, z)
     assert B.paro_fault_status() == 0
 
 

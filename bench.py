@@ -59,9 +59,25 @@ def call_bytes(T, n_in, n_out):
 
 # DRAM bytes (read + write) per decode-kernel launch, mean over the four
 # projections (qkv 13.24 MB, o 8.89 MB, gate+up 61.18 MB, down 31.00 MB), from
-# one ncu capture of the current kernel at 16 tokens; the command is in
-# profiles/gemv_kernel_gate_up_4096x28672_t16.md. None once the kernel changes.
+# one ncu capture at 16 tokens of the decode kernel built from the gemv.cu
+# whose SHA-256 prefix is GEMV_TRAFFIC_SOURCE; reported only while gemv.cu is
+# that file (any change to it nulls the figure until it is captured again).
 GEMV_TRAFFIC_PER_LAUNCH_T16 = (13238528 + 8886272 + 61180416 + 30999040) / 4
+GEMV_TRAFFIC_SOURCE = "unset"
+
+
+def gemv_source_sha() -> str:
+    import hashlib
+    with open(os.path.join(ROOT, "rotated_w4_linear_b200", "csrc", "gemv.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def gemv_traffic(tokens: int, model: str):
+    """The captured DRAM traffic per decode launch, if it belongs to this
+    workload and to the current kernel source; else None."""
+    if tokens != 16 or model != "llama3-8b" or gemv_source_sha() != GEMV_TRAFFIC_SOURCE:
+        return None
+    return GEMV_TRAFFIC_PER_LAUNCH_T16
 
 
 def peaks():
@@ -152,9 +168,9 @@ def decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_byte
         "config": config(args),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
-                     "traffic": (GEMV_TRAFFIC_PER_LAUNCH_T16
-                                 if args.tokens == 16 and args.model == "llama3-8b" else None),
-                     "kernel": "gemv_kernel (int4 decode)",
+                     "traffic": gemv_traffic(args.tokens, args.model),
+                     "kernel": "gemv_kernel (int4 decode; timed on unrotated inputs, the branch that "
+                               "reads X in natural order)",
                      "us_per_launch": 1e6 * kern_s / (args.steps * n_calls),
                      "peak_source": f"{peak_kind} hbm_gbs"},
         "e2e": {"value": step_bytes * args.steps * world / e2e_elapsed / 1e9, "unit": "GB/s",
@@ -252,12 +268,12 @@ def config(args):
 
 
 # --------------------------------------------------------------------------- rotation alone
-def bench_rotate(args, torch, B, local):
-    """paro_rotate on X [tokens][4096] (fp16 in, fp16 out), distinct inputs per
-    call so that each step moves more than L2. Bytes: X read + X' written +
-    rotation parameters."""
+def rotate_result(torch, B, local, T, K, P, steps, warmup, n_in=4096):
+    """paro_rotate on X [T][n_in] (fp16 in, fp16 out), distinct inputs per
+    call so that each pass moves more than L2, replayed from a CUDA graph.
+    Algorithmic bytes: X read + X' written + the rotation parameters
+    (per pair an fp32 cos/sin pair and two channel bytes, plus 1/alpha)."""
     torch.cuda.set_device(local)
-    T, n_in, K, P = args.tokens, 4096, args.rot_k, args.rot_pairs
     pairs, theta, alpha = synth.rotation_params(n_in, K, synth.layer_seed(1, K), pairs_per_group=P)
     rot = B.paro_rot_create(pairs, theta, alpha)
     copies = min(64, max(1, (512 << 20) // (4 * T * n_in)))   # > L2 for T >= 256
@@ -273,40 +289,48 @@ def bench_rotate(args, torch, B, local):
     with torch.cuda.graph(g):
         for x, y in zip(xs, ys):
             B.paro_rotate(rot, x, y)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-    per = e0.elapsed_time(e1) / 1e3 / (args.steps * len(xs))
+    per = e0.elapsed_time(e1) / 1e3 / (steps * len(xs))
     del g
+    rot.close()
     nbytes = 4 * T * n_in + K * (n_in // GROUP) * P * 10 + 4 * n_in
     hbm_peak, _, kind = peaks()
-    print(json.dumps({"workload": f"paro_rotate tokens={T} hidden={n_in} K={K} pairs/group={P}",
-                      "us_per_call": per * 1e6, "GB/s": nbytes / per / 1e9,
-                      "roofline": {"bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm_peak,
-                                   "frac": nbytes / per / 1e9 / hbm_peak, "peak_source": kind},
-                      "copies": copies, "clocks": clk.summary()}), flush=True)
+    kern = "rotate_tc_kernel (tensor cores)" if T >= 128 else "rotate_kernel / rotate_quad_kernel (Givens)"
+    return {"workload": f"paro_rotate tokens={T} hidden={n_in} K={K} pairs/group={P}",
+            "us_per_call": per * 1e6, "GB/s": nbytes / per / 1e9,
+            "roofline": {"bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": nbytes / per / 1e9 / hbm_peak, "traffic": None, "kernel": kern,
+                         "bytes_per_call": nbytes, "peak_source": f"{kind} hbm_gbs"},
+            "copies": copies, "l2": "inputs larger than L2 (distinct copies per pass)" if 4 * T * n_in * copies > 126e6
+            else "inputs smaller than L2", "clocks": clk.summary()}
+
+
+def bench_rotate(args, torch, B, local):
+    print(json.dumps(rotate_result(torch, B, local, args.tokens, args.rot_k, args.rot_pairs, args.steps,
+                                   args.warmup)), flush=True)
     return 0
 
 
 # --------------------------------------------------------------------------- prefill
-def bench_prefill(args, torch, B, local):
-    """One Llama-3-8B-shaped layer's projections at --tokens: rotation +
+def prefill_result(torch, B, local, T, steps, warmup, model):
+    """One decoder layer's projections (`model` shapes) at T tokens: rotation +
     tensor-core GEMM per projection, replayed as a CUDA graph. Reports the
     GEMM FLOP rate (2 T in out per projection) against the measured dense
     16-bit tensor peak, and the rotation overhead against the same GEMMs on
     unrotated inputs (theta = 0, alpha = 1: no rotation launch)."""
     torch.cuda.set_device(local)
-    T = args.tokens
     dev = torch.device("cuda", local)
     calls = []
-    for i, (name, n_in, n_out) in enumerate(PROJ):
+    for i, (name, n_in, n_out) in enumerate(MODELS[model]):
         seed = synth.layer_seed(3, i)
         pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
         rot = B.paro_rot_create(pairs, theta, alpha)
@@ -331,7 +355,7 @@ def bench_prefill(args, torch, B, local):
         with torch.cuda.graph(g):
             step(rot)
         graphs[rot] = g
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         graphs[True].replay(); graphs[False].replay()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -340,11 +364,11 @@ def bench_prefill(args, torch, B, local):
         for rot in (True, False):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for _ in range(args.steps):
+            for _ in range(steps):
                 graphs[rot].replay()
             e1.record(stream)
             torch.cuda.synchronize()
-            times[rot] = e0.elapsed_time(e1) / 1e3 / args.steps
+            times[rot] = e0.elapsed_time(e1) / 1e3 / steps
     flops = sum(2.0 * T * p["n_in"] * p["n_out"] for p in calls)
     _, _, kind = peaks()
     try:
@@ -353,17 +377,24 @@ def bench_prefill(args, torch, B, local):
     except Exception:
         tc_peak = 1400.0
     tf = flops / times[False] / 1e12
-    print(json.dumps({"workload": f"prefill {args.model} layer projections, {T} tokens, K={K_LAYERS}",
-                      "ms_per_layer": 1e3 * times[True], "ms_per_layer_unrotated": 1e3 * times[False],
-                      "TFLOP/s": flops / times[True] / 1e12, "TFLOP/s_gemm_only": tf,
-                      "rotation_overhead": times[True] / times[False] - 1.0,
-                      "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
-                                   "frac": tf / tc_peak, "peak_source": f"{kind} bf16_tflops_sustained "
-                                   "(fp16 and bf16 share the dense tensor rate)"},
-                      "clocks": clk.summary()}), flush=True)
+    shapes = ", ".join(f"{n} {i}x{o}" for n, i, o in MODELS[model])
+    res = {"workload": f"prefill {model} decoder-layer projections ({shapes}), {T} tokens, K={K_LAYERS}",
+           "ms_per_layer": 1e3 * times[True], "ms_per_layer_unrotated": 1e3 * times[False],
+           "TFLOP/s": flops / times[True] / 1e12, "TFLOP/s_gemm_only": tf,
+           "rotation_overhead": times[True] / times[False] - 1.0,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
+                        "frac": tf / tc_peak, "traffic": None, "kernel": "gemm_w4_kernel (tcgen05)",
+                        "flops_per_layer": flops,
+                        "peak_source": f"{kind} bf16_tflops_sustained (fp16 and bf16 share the dense tensor rate)"},
+           "l2": "inputs larger than L2", "clocks": clk.summary()}
     del graphs
     for p in calls:
         p["rot"].close()
+    return res
+
+
+def bench_prefill(args, torch, B, local):
+    print(json.dumps(prefill_result(torch, B, local, args.tokens, args.steps, args.warmup, args.model)), flush=True)
     return 0
 
 
@@ -377,6 +408,8 @@ def main():
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--impl", default="paro", choices=["paro", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the rotation and prefill figures that the decode line carries by default")
     ap.add_argument("--workload", default="decode", choices=["decode", "rotate", "prefill"],
                     help="decode: the headline step; rotate: paro_rotate alone (hidden 4096); "
                          "prefill: one layer's projections at --tokens (tensor-core GEMM)")
@@ -571,13 +604,24 @@ def main():
     elapsed, e2e_elapsed, kern_s = max_over_ranks(dist, [elapsed, e2e_elapsed, kern_s], dev)
     line = decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_bytes, len(calls),
                        hbm_peak, peak_kind, h2d, d2h, per_proj, n_launch, clocks)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(T)
-    emit(line, rank)
     del g_step, g_gemv
     for projs in layers:
         for p in projs:
             p["rot"].close()
+    del layers, calls, sets
+    torch.cuda.empty_cache()
+    # the other two kernels of the path, in the same run: the rotation alone
+    # (paro_rotate on [8192 x 4096], K = 8) and one prefill layer at 8192
+    # tokens (tensor-core GEMM, with the rotation overhead); every rank runs
+    # them on its own GPU, rank 0 reports its figures
+    if not args.no_extra:
+        xs = min(args.steps, 20)
+        line["rotate"] = rotate_result(torch, B, local, 8192, K_LAYERS, 64, xs, 3)
+        line["prefill"] = prefill_result(torch, B, local, 8192, xs, 3, args.model)
+        torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(T)
+    emit(line, rank)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

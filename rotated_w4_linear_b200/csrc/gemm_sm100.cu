@@ -279,7 +279,6 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 // host side
 // ---------------------------------------------------------------------------
 namespace {
-
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {  // driver entry point, no link-time libcuda
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -292,6 +291,23 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {  // driver entry point, no lin
     });
     return fn;
 }
+
+}  // namespace
+
+bool encode_tma_2d(CUtensorMap* tm, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(tm, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
+namespace {
 
 template <int BN, int STAGES, int DQG, int NACC>
 cudaError_t launch_cfg(const CUtensorMap* tm, const GemmArgs& a, int mt, int nt, cudaStream_t s) {
@@ -332,31 +348,19 @@ cudaError_t launch_cfg(const CUtensorMap* tm, const GemmArgs& a, int mt, int nt,
     return cudaLaunchKernelEx(&cfg, gemm_w4_kernel<BN, STAGES, DQG, NACC>, tm[0], tm[1], tm[2], tm[3], a);
 }
 
-bool encode_2d(CUtensorMap* tm, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
-               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1u, 1u};
-    return enc(tm, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // tm[0]: X' [T][in] fp16, box 64 channels x BN tokens, 128-byte swizzle, zero fill past T
 // tm[1]: packed int4 codes as uint32 [out/16][in/64 * 128], box one k block x 8 row blocks
 // tm[2]: scales uint32 [out/16][G * 8], box one group x 8 row blocks
 // tm[3]: zeros uint8 [out/16][Gp * 8], box two groups x 8 row blocks
 bool encode_maps(const void* Xr, const void* qw, const void* sp, const void* zp, int64_t T, int BN,
                  const GemmArgs& a, CUtensorMap* tm) {
-    return encode_2d(&tm[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xr, (uint64_t)a.in, (uint64_t)T, (uint64_t)a.in * 2,
+    return encode_tma_2d(&tm[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xr, (uint64_t)a.in, (uint64_t)T, (uint64_t)a.in * 2,
                      64u, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-           encode_2d(&tm[1], CU_TENSOR_MAP_DATA_TYPE_UINT32, qw, (uint64_t)a.nkb * 128, (uint64_t)a.nrb,
+           encode_tma_2d(&tm[1], CU_TENSOR_MAP_DATA_TYPE_UINT32, qw, (uint64_t)a.nkb * 128, (uint64_t)a.nrb,
                      (uint64_t)a.nkb * 512, 128u, 8u, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-           encode_2d(&tm[2], CU_TENSOR_MAP_DATA_TYPE_UINT32, sp, (uint64_t)a.G * 8, (uint64_t)a.nrb,
+           encode_tma_2d(&tm[2], CU_TENSOR_MAP_DATA_TYPE_UINT32, sp, (uint64_t)a.G * 8, (uint64_t)a.nrb,
                      (uint64_t)a.G * 32, 8u, 8u, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-           encode_2d(&tm[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, zp, (uint64_t)a.Gp * 8, (uint64_t)a.nrb,
+           encode_tma_2d(&tm[3], CU_TENSOR_MAP_DATA_TYPE_UINT8, zp, (uint64_t)a.Gp * 8, (uint64_t)a.nrb,
                      (uint64_t)a.Gp * 8, 16u, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 

@@ -1,6 +1,7 @@
 // Host-side launchers of the sm_100a kernels (internal to libparo).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,9 +17,19 @@ struct RotDev {
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha
     uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
     double* alpha64 = nullptr;     // [in] alpha as fp64
+    uint8_t* mats = nullptr;       // [G][64 KB] dense per-group rotation (hi, lo fp16; tensor-core operand image)
 };
 
+// Bytes of one group's dense rotation image: hi and lo fp16 128 x 128.
+constexpr size_t kRotMatBytes = 4 * 128 * 128;
+
+// 2-D TMA descriptor of a row-major tensor [outer][inner] (driver entry point).
+bool encode_tma_2d(CUtensorMap* tm, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
+// Tensor-core rotation (dense per-group matrices); any T >= 1.
+cudaError_t launch_rotate_tc(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
 // Decode batches (1 <= T <= 16): one CTA per group, all layers' parameters in
 // shared memory; launched as a programmatic dependent of the previous kernel.
 // lane_major: X' is written with every 64-channel block in the decode

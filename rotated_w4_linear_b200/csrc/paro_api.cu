@@ -60,6 +60,41 @@ paro_status check_shape(int64_t in, int64_t out) {
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
+// Dense form of one group's activation rotation: M = diag(1/alpha) R_1^T ...
+// R_K^T (x' = x M for a row x of the group's 128 channels), built in fp64 by
+// applying the layers, in order, to every row of diag(1/alpha) with the 2x2
+// formula. Written as the tensor-core B operand image (rotate_tc.cu): B[n][k]
+// = M[k][n] for hi = fp16(M) and then lo = fp16(M - hi), each as two halves
+// (k 0-63, 64-127) of 128 rows x 128 bytes, 16-byte chunk c of row n at chunk
+// position c ^ (n mod 8) (the 128-byte swizzle of a K-major operand).
+void dense_group_image(const int16_t* pairs, const float* theta, const float* alpha, int K, int P, int G, int g,
+                       uint8_t* out) {
+    std::vector<double> M(128 * 128, 0.0);                // M[k * 128 + n]
+    for (int k = 0; k < 128; ++k) M[k * 128 + k] = 1.0 / (double)alpha[g * 128 + k];
+    for (int t = 0; t < K; ++t)
+        for (int p = 0; p < P; ++p) {
+            const size_t base = (((size_t)t * G + g) * P + p);
+            const int i = pairs[2 * base], j = pairs[2 * base + 1];
+            const double c = std::cos((double)theta[base]), sn = std::sin((double)theta[base]);
+            for (int k = 0; k < 128; ++k) {
+                const double vi = M[k * 128 + i], vj = M[k * 128 + j];
+                M[k * 128 + i] = c * vi - sn * vj;
+                M[k * 128 + j] = sn * vi + c * vj;
+            }
+        }
+    for (int part = 0; part < 2; ++part)
+        for (int n = 0; n < 128; ++n)
+            for (int k = 0; k < 128; ++k) {
+                const double m = M[k * 128 + n];
+                const __half hi = __double2half(m);
+                const __half v = part == 0 ? hi : __double2half(m - (double)__half2float(hi));
+                const int h = k >> 6, chunk = (k & 63) >> 3, e = k & 7;
+                const size_t off = (size_t)part * 32768 + (size_t)h * 16384 + (size_t)n * 128 +
+                                   (size_t)((chunk ^ (n & 7)) << 4) + (size_t)e * 2;
+                memcpy(out + off, &v, 2);
+            }
+}
+
 // Plain host memory (not allocated or registered with CUDA) that a kernel
 // cannot read.
 bool is_unregistered_host(const void* p) {
@@ -271,6 +306,9 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
             }
         }
     }
+    // dense per-group rotations for the tensor-core kernel
+    std::vector<uint8_t> mats((size_t)G * paro::kRotMatBytes);
+    for (int g = 0; g < G; ++g) dense_group_image(pairs, theta, alpha, K, P, G, g, &mats[(size_t)g * paro::kRotMatBytes]);
     std::vector<float> inv_alpha((size_t)in);
     std::vector<double> alpha64((size_t)in);
     for (int64_t c = 0; c < in; ++c) {
@@ -283,7 +321,8 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     const size_t o_a64 = o_rot64 + round256(rot64.size());
     const size_t o_rotx = o_a64 + round256(alpha64.size() * sizeof(double));
     const size_t o_rotq = o_rotx + round256(rotx.size());
-    const size_t total = o_rotq + round256(rotq.size());
+    const size_t o_mats = o_rotq + round256(rotq.size());
+    const size_t total = o_mats + round256(mats.size());
 
     paro_rot* r = new (std::nothrow) paro_rot();
     if (!r) return fail(PARO_ERR_ARG, "out of host memory");
@@ -296,6 +335,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !rotx.empty()) e = cudaMemcpy(base + o_rotx, rotx.data(), rotx.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !rotq.empty()) e = cudaMemcpy(base + o_rotq, rotq.data(), rotq.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + o_mats, mats.data(), mats.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { cudaFree(r->block); delete r; return cuda_fail(e, "cudaMemcpy(rotation tables)"); }
     r->dev.in = in;
     r->dev.G = G;
@@ -306,6 +346,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);
     r->dev.rotx = reinterpret_cast<uint8_t*>(base + o_rotx);
     r->dev.rotq = reinterpret_cast<uint8_t*>(base + o_rotq);
+    r->dev.mats = reinterpret_cast<uint8_t*>(base + o_mats);
     *out = r;
     return PARO_OK;
 }

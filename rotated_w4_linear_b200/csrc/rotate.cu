@@ -315,6 +315,9 @@ namespace {
 // decode batches (T <= 16): one CTA per group, one warp per quad;
 // larger batches: 8 warps of QW_BIG quads (4 QW_BIG tokens) per CTA
 constexpr int QW_BIG = 2;
+// from this many tokens on the tensor-core kernel (rotate_tc.cu) rotates:
+// its per-group matrices (64 KB each) then cost less than the activations
+constexpr int64_t kRotateTcMinTokens = 128;
 
 template <int QW, bool PF>
 cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int warps, cudaStream_t s,
@@ -387,7 +390,7 @@ cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, c
     const __half* x = static_cast<const __half*>(X);
     __half* y = static_cast<__half*>(Xr);
     if (T <= 16) return launch_rotate_decode(r, X, Xr, T, s);
-    if (T >= 256) return launch_quad<QW_BIG, true>(r, X, Xr, T, 8, s, 0);
+    if (T >= kRotateTcMinTokens) return launch_rotate_tc(r, X, Xr, T, s);
     const cudaError_t e = launch_rotate_t<8>(r, x, y, T, s);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -78,10 +78,23 @@ def test_decode_line_carries_every_contract_key():
         assert k in line["roofline"], k
     for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
         assert k in line["e2e"], k
-    assert line["roofline"]["traffic"] == bench.GEMV_TRAFFIC_PER_LAUNCH_T16
+    # the captured traffic belongs to one kernel source: reported only while
+    # gemv.cu is that file
+    want = bench.GEMV_TRAFFIC_PER_LAUNCH_T16 if bench.gemv_source_sha() == bench.GEMV_TRAFFIC_SOURCE else None
+    assert line["roofline"]["traffic"] == want
     assert line["e2e"]["value"] == pytest.approx(1e9 * 10 / 3.0 / 1e9)
     json.dumps(line)
     # the measured traffic belongs to one workload: no figure for another one
     other = types.SimpleNamespace(**{**vars(args), "model": "qwen3-4b"})
     assert bench.decode_line(other, 1, 2.0, 3.0, 1.0, 1e9, 5e8, 16, 6454.9, "measured", 1, 2, {}, 320,
                              {})["roofline"]["traffic"] is None
+
+
+def test_traffic_figure_follows_the_kernel_source(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(bench, "GEMV_TRAFFIC_SOURCE", bench.gemv_source_sha())
+    assert bench.gemv_traffic(16, "llama3-8b") == bench.GEMV_TRAFFIC_PER_LAUNCH_T16
+    assert bench.gemv_traffic(4, "llama3-8b") is None
+    monkeypatch.setattr(bench, "GEMV_TRAFFIC_SOURCE", "0" * 16)
+    assert bench.gemv_traffic(16, "llama3-8b") is None

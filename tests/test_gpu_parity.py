@@ -66,11 +66,12 @@ def test_rotate_parity(B, T, in_f, K, P):
 
 
 @pytest.mark.parametrize("in_f,K,P", [(4096, 8, 64), (14336, 16, 13), (384, 3, 64)])
-def test_rotate_kernels_agree_bit_for_bit(B, in_f, K, P):
-    """Batches of at most 16 tokens and of 256 or more take the quad kernel
-    (float4 exchange, packed f32x2 arithmetic; from 9 tokens on with each
-    layer's tables loaded during the layer before); the others the general
-    one. All apply the same operations in the same order: identical bits."""
+def test_rotate_givens_kernels_agree_bit_for_bit(B, in_f, K, P):
+    """Batches of at most 16 tokens take the quad kernel (float4 exchange,
+    packed f32x2 arithmetic; from 9 tokens on with each layer's tables loaded
+    during the layer before), 17 to 127 tokens the general one. Both apply
+    the Givens layers with the same operations in the same order: identical
+    bits."""
     seed = synth.layer_seed(1, 77 + K)
     pairs, theta, alpha = synth.rotation_params(in_f, K, seed, pairs_per_group=P)
     x = synth.activations(24, in_f, seed)
@@ -79,13 +80,38 @@ def test_rotate_kernels_agree_bit_for_bit(B, in_f, K, P):
     for T in (1, 7, 8, 9, 16):
         small = host(B.paro_rotate(rot, dev(x[:T])))
         assert np.array_equal(small.view(np.uint16), big[:T].view(np.uint16)), T
-    check_rotation(big[:16], x[:16], pairs, theta, alpha)
-    # batches of 256 tokens and more take the quad kernel with several quads per warp
-    x2 = synth.activations(300, in_f, seed + 1)
-    general = host(B.paro_rotate(rot, dev(x2[:255])))
-    quad = host(B.paro_rotate(rot, dev(x2)))
-    assert np.array_equal(quad[:255].view(np.uint16), general.view(np.uint16))
-    check_rotation(quad, x2, pairs, theta, alpha)
+    check_rotation(big, x, pairs, theta, alpha)
+
+
+@pytest.mark.parametrize("T,in_f,K,P", [
+    (128, 384, 8, 64),      # one 128-token tile, three groups
+    (129, 4096, 8, 64),     # ragged second tile
+    (300, 256, 1, 64),      # one layer: a sparse M
+    (300, 384, 4, 13),      # partial matchings
+    (1000, 4096, 16, 64),   # sixteen layers
+    (777, 640, 0, 1),       # K = 0: M = diag(1/alpha)
+    (2048, 14336, 8, 64),   # down-projection width: 112 groups
+])
+def test_rotate_tensor_core_parity(B, T, in_f, K, P):
+    """From 128 tokens on, each group's diag(1/alpha) R_1^T .. R_K^T is applied
+    as one dense matrix on the tensor cores (fp16 hi + lo parts, fp32
+    accumulation): every element against the fp64 oracle."""
+    seed = synth.layer_seed(1, 500 + T + K)
+    pairs, theta, alpha = synth.rotation_params(in_f, max(K, 1), seed, pairs_per_group=P)
+    if K == 0:
+        pairs, theta = pairs[:0], theta[:0]
+    x = synth.activations(T, in_f, seed)
+    rot = B.paro_rot_create(pairs, theta, alpha)
+    got = host(B.paro_rotate(rot, dev(x)))
+    if T * in_f > 4_000_000:                           # large: sampled rows, first and last included
+        rows = np.unique(np.concatenate([[0, T - 1], np.random.default_rng(T).choice(T, 96, replace=False)]))
+        check_rotation(got[rows], x[rows], pairs, theta, alpha)
+    else:
+        check_rotation(got, x, pairs, theta, alpha)
+    assert B.paro_fault_status() == 0
+    # a row's result does not depend on the batch or the tile it is in
+    twice = host(B.paro_rotate(rot, dev(np.concatenate([x[T // 3:], x]))))
+    assert np.array_equal(twice[T - T // 3:].view(np.uint16), got.view(np.uint16))
 
 
 @pytest.mark.parametrize("T", [2048, 8192])

@@ -10,7 +10,7 @@ namespace paro {
 
 // ---------------------------------------------------------------------------
 // Prepared rotation parameters ("rotation block", host image from which the
-// device exchange blocks below are built), one per (layer t, group g), 1152
+// quad exchange blocks below are built), one per (layer t, group g), 1152
 // bytes: 128 partner bytes, then 128 float2 (a, b).
 // Channel c of the group becomes a * v[c] + b * v[partner[c]]:
 //   first channel i of a pair (i, j, th): a = cos th, b = -sin th, partner j
@@ -20,24 +20,6 @@ namespace paro {
 // written per output channel.
 // ---------------------------------------------------------------------------
 constexpr int kRotBlockBytes = 128 + 128 * 8;
-
-// ---------------------------------------------------------------------------
-// Exchange blocks for the rotation kernel, one per (layer t, group g), 1536 B:
-//   [32 lanes][uint4]: byte offsets (u16) in the warp's 512-byte exchange row
-//     where lane L stores its channels 4L..4L+3 (x: w0|w1<<16, y: w2|w3<<16)
-//     and where it loads their partners (z: r0|r1<<16, w: r2|r3<<16);
-//   [128 channels][float2]: (a, b) as in the rotation block.
-// The host chooses the positions so that each of the four stores and each of
-// the four loads of a warp hits 32 distinct banks: writes grouped by the slot
-// of the channel and reads grouped by the slot of its partner form a 4 x 4
-// bipartite multigraph with every node of degree 32, whose edges are coloured
-// with 32 colours (Koenig's theorem); the colour is the bank.
-// ---------------------------------------------------------------------------
-constexpr int kRotXBlockBytes = 32 * 16 + 128 * 8;
-
-__device__ __forceinline__ const uint8_t* rotx_block(const uint8_t* rotx, int t, int g, int G) {
-    return rotx + ((size_t)t * G + g) * kRotXBlockBytes;
-}
 
 // ---------------------------------------------------------------------------
 // Quad exchange blocks for the decode rotation kernel, one per

@@ -12,7 +12,6 @@ struct RotDev {
     int G = 0;              // groups of 128
     int K = 0;              // rotation layers
     int P = 0;              // active pairs per (layer, group)
-    uint8_t* rotx = nullptr;       // [K][G] exchange blocks: conflict-free positions + coefficients
     uint8_t* rotq = nullptr;       // [K][G] quad exchange blocks (decode prologue)
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha
     uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
@@ -30,6 +29,7 @@ bool encode_tma_2d(CUtensorMap* tm, CUtensorMapDataType type, const void* base, 
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
 // Tensor-core rotation (dense per-group matrices); any T >= 1.
 cudaError_t launch_rotate_tc(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s);
+// X' = X T^-1: Givens kernel up to 16 tokens, tensor-core kernel above.
 // Decode batches (1 <= T <= 16): one CTA per group, all layers' parameters in
 // shared memory; launched as a programmatic dependent of the previous kernel.
 // lane_major: X' is written with every 64-channel block in the decode

@@ -211,44 +211,6 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
             }
         }
     }
-    // exchange blocks: bank-conflict-free positions (edge colouring) + coefficients
-    std::vector<uint8_t> rotx((size_t)K * G * paro::kRotXBlockBytes);
-    for (int t = 0; t < K; ++t) {
-        for (int g = 0; g < G; ++g) {
-            const uint8_t* b = &rot32[((size_t)t * G + g) * paro::kRotBlockBytes];
-            const uint8_t* partner = b;
-            // buckets[i][j]: channels c with c % 4 == i (store slot) and partner % 4 == j (load slot)
-            std::vector<int> buckets[4][4];
-            for (int c = 0; c < 128; ++c) buckets[c & 3][partner[c] & 3].push_back(c);
-            int pos[128];
-            int used_rows[32] = {0};
-            for (int color = 0; color < 32; ++color) {
-                int perm[4] = {0, 1, 2, 3};
-                bool found = false;
-                do {
-                    bool ok = true;
-                    for (int i = 0; i < 4 && ok; ++i) ok = !buckets[i][perm[i]].empty();
-                    if (ok) { found = true; break; }
-                } while (std::next_permutation(perm, perm + 4));
-                if (!found) return fail(PARO_ERR_ARG, "internal: no conflict-free exchange layout");
-                for (int i = 0; i < 4; ++i) {
-                    const int c = buckets[i][perm[i]].back();
-                    buckets[i][perm[i]].pop_back();
-                    pos[c] = color + 32 * used_rows[color]++;
-                }
-            }
-            uint8_t* x = &rotx[((size_t)t * G + g) * paro::kRotXBlockBytes];
-            for (int l = 0; l < 32; ++l) {
-                uint16_t o[8];
-                for (int r = 0; r < 4; ++r) {
-                    o[r] = (uint16_t)(4 * pos[4 * l + r]);
-                    o[4 + r] = (uint16_t)(4 * pos[partner[4 * l + r]]);
-                }
-                memcpy(x + 16 * l, o, 16);
-            }
-            memcpy(x + 512, b + 128, 1024);
-        }
-    }
     // quad exchange blocks: 16-byte slots, 8 lanes of a quarter-warp on 8 distinct
     // slots mod 8 for every store and load (8 perfect matchings of an 8-regular
     // bipartite multigraph, found one after another by augmenting paths)
@@ -319,8 +281,7 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     const size_t o_inv = 0;
     const size_t o_rot64 = o_inv + round256(inv_alpha.size() * sizeof(float));
     const size_t o_a64 = o_rot64 + round256(rot64.size());
-    const size_t o_rotx = o_a64 + round256(alpha64.size() * sizeof(double));
-    const size_t o_rotq = o_rotx + round256(rotx.size());
+    const size_t o_rotq = o_a64 + round256(alpha64.size() * sizeof(double));
     const size_t o_mats = o_rotq + round256(rotq.size());
     const size_t total = o_mats + round256(mats.size());
 
@@ -333,7 +294,6 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     e = cudaMemcpy(base + o_inv, inv_alpha.data(), inv_alpha.size() * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_rot64, rot64.data(), rot64.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess && !rotx.empty()) e = cudaMemcpy(base + o_rotx, rotx.data(), rotx.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !rotq.empty()) e = cudaMemcpy(base + o_rotq, rotq.data(), rotq.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(base + o_mats, mats.data(), mats.size(), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { cudaFree(r->block); delete r; return cuda_fail(e, "cudaMemcpy(rotation tables)"); }
@@ -344,7 +304,6 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     r->dev.inv_alpha = reinterpret_cast<float*>(base + o_inv);
     r->dev.rotp64 = reinterpret_cast<uint8_t*>(base + o_rot64);
     r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);
-    r->dev.rotx = reinterpret_cast<uint8_t*>(base + o_rotx);
     r->dev.rotq = reinterpret_cast<uint8_t*>(base + o_rotq);
     r->dev.mats = reinterpret_cast<uint8_t*>(base + o_mats);
     *out = r;

@@ -1,117 +1,20 @@
-// Activation rotation X' = X T^-1 (ParoQuant CSDN article, section 2.1; the
-// online rotation kernel of section 3.1): per token row and 128-channel group,
-// divide by alpha, then K layers of independent Givens pairs, fp32 in
-// registers, fp16 out.
+// Activation rotation X' = X T^-1 with the Givens layers themselves, for
+// decode batches of at most 16 tokens (ParoQuant CSDN article, section 2.1;
+// the online rotation kernel of section 3.1): per token row and 128-channel
+// group, divide by alpha, then K layers of independent Givens pairs, fp32 in
+// registers, fp16 out. Larger batches go to the tensor-core kernel
+// (rotate_tc.cu), which applies each group's whole rotation as one matrix.
 //
-// Mapping: one warp owns one (group, token tile). Lane L holds channels
-// 4L..4L+3 of TT tokens, loaded as one 8-byte vector per token (a warp reads
-// 256 contiguous bytes per row). Partner values are exchanged through a
-// warp-private shared-memory row per token each layer, at positions chosen on
-// the host so that every store and load is bank-conflict-free; the next
-// layer's positions and coefficients are loaded while the current one runs.
+// Mapping: one CTA per group, one warp per quad of four tokens. Lane L holds
+// channels 4L..4L+3 of the quad; partner values are exchanged through a
+// warp-private shared-memory buffer each layer, at positions chosen on the
+// host so that every access is bank-conflict-free.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
 
 namespace paro {
-
-template <int TT>
-__global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ X, __half* __restrict__ Xr,
-                                                     int64_t T, int in, int G, int K,
-                                                     const uint8_t* __restrict__ rotx,
-                                                     const float* __restrict__ inv_alpha) {
-    // a kernel launched after this one on the stream may start now; it waits
-    // for this grid's completion before it reads Xr
-    asm volatile("griddepcontrol.launch_dependents;");
-    // this kernel is itself a programmatic dependent launch: X may be the
-    // output of the kernel before it, so X is read only after this wait
-    // (the rotation parameters are never written by a kernel on the path)
-    __shared__ __align__(16) float buf[4][TT][128];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t task = (int64_t)blockIdx.x * 4 + warp;
-    const int g = (int)(task % G);
-    const int64_t t0 = (task / G) * TT;
-    if (t0 >= T) return;
-    const int c0 = g * 128 + 4 * lane;
-
-    const float4 ia = __ldg(reinterpret_cast<const float4*>(inv_alpha + c0));
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    float v[TT][4];
-#pragma unroll
-    for (int i = 0; i < TT; ++i) {
-        uint2 raw = make_uint2(0u, 0u);
-        if (t0 + i < T) raw = __ldg(reinterpret_cast<const uint2*>(X + (t0 + i) * in + c0));
-        const float2 lo = __half22float2(*reinterpret_cast<__half2*>(&raw.x));
-        const float2 hi = __half22float2(*reinterpret_cast<__half2*>(&raw.y));
-        v[i][0] = lo.x * ia.x;
-        v[i][1] = lo.y * ia.y;
-        v[i][2] = hi.x * ia.z;
-        v[i][3] = hi.y * ia.w;
-    }
-
-    // Each layer: every lane stores its 4 channels at the layer's positions
-    // in the warp's exchange rows (one 512-byte row per token), then loads
-    // the 4 partners; positions make every access bank-conflict-free.
-    float* row0 = &buf[warp][0][0];
-    uint4 off = make_uint4(0u, 0u, 0u, 0u);
-    float4 c01 = make_float4(1.f, 0.f, 1.f, 0.f), c23 = c01;
-    if (K > 0) {
-        const uint8_t* blk = rotx_block(rotx, 0, g, G);
-        off = __ldg(reinterpret_cast<const uint4*>(blk) + lane);
-        c01 = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane);
-        c23 = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane + 1);
-    }
-    for (int t = 0; t < K; ++t) {
-        uint4 off_n = off;
-        float4 c01_n = c01, c23_n = c23;
-        if (t + 1 < K) {                                   // next layer's parameters in flight
-            const uint8_t* blk = rotx_block(rotx, t + 1, g, G);
-            off_n = __ldg(reinterpret_cast<const uint4*>(blk) + lane);
-            c01_n = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane);
-            c23_n = __ldg(reinterpret_cast<const float4*>(blk + 512) + 2 * lane + 1);
-        }
-        // byte offsets -> float indices into the token-0 row; token i adds 128 i
-        float* w0 = row0 + ((off.x & 0xFFFFu) >> 2);
-        float* w1 = row0 + (off.x >> 18);
-        float* w2 = row0 + ((off.y & 0xFFFFu) >> 2);
-        float* w3 = row0 + (off.y >> 18);
-        const float* r0 = row0 + ((off.z & 0xFFFFu) >> 2);
-        const float* r1 = row0 + (off.z >> 18);
-        const float* r2 = row0 + ((off.w & 0xFFFFu) >> 2);
-        const float* r3 = row0 + (off.w >> 18);
-#pragma unroll
-        for (int i = 0; i < TT; ++i) {
-            w0[i * 128] = v[i][0];
-            w1[i * 128] = v[i][1];
-            w2[i * 128] = v[i][2];
-            w3[i * 128] = v[i][3];
-        }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < TT; ++i) {
-            const float q0 = r0[i * 128], q1 = r1[i * 128], q2 = r2[i * 128], q3 = r3[i * 128];
-            v[i][0] = fmaf(c01.y, q0, c01.x * v[i][0]);
-            v[i][1] = fmaf(c01.w, q1, c01.z * v[i][1]);
-            v[i][2] = fmaf(c23.y, q2, c23.x * v[i][2]);
-            v[i][3] = fmaf(c23.w, q3, c23.z * v[i][3]);
-        }
-        __syncwarp();
-        off = off_n;
-        c01 = c01_n;
-        c23 = c23_n;
-    }
-
-#pragma unroll
-    for (int i = 0; i < TT; ++i) {
-        if (t0 + i < T) {
-            uint2 o;
-            o.x = pack_half2(v[i][0], v[i][1]);
-            o.y = pack_half2(v[i][2], v[i][3]);
-            *reinterpret_cast<uint2*>(Xr + (t0 + i) * in + c0) = o;
-        }
-    }
-}
 
 // Quad kernel. Work items are (128-channel group g, token tile) in
 // group-major order, a tile being nw warps x QW quads of four tokens; CTA c
@@ -126,7 +29,7 @@ __global__ void __launch_bounds__(128) rotate_kernel(const __half* __restrict__ 
 // packed f32x2 multiply and fma. With QW > 1 each warp uses two 2 KB
 // exchange buffers alternately (one warp barrier per quad and layer) and
 // loads the next item's X while it rotates the current one. The operations
-// and their order are those of rotate_kernel, so X' is bit-identical.
+// and their order do not depend on the batch, so a row's X' does not either.
 // PF: each layer's table entries are loaded during the layer before.
 // lane_major != 0 writes each 64-channel block of X' in the order the decode
 // kernel's B fragments read it: channel 16 j + 4 q + e at position
@@ -312,12 +215,9 @@ __global__ void __launch_bounds__(256) rotate_quad_kernel(const __half* __restri
 
 namespace {
 
-// decode batches (T <= 16): one CTA per group, one warp per quad;
-// larger batches: 8 warps of QW_BIG quads (4 QW_BIG tokens) per CTA
-constexpr int QW_BIG = 2;
-// from this many tokens on the tensor-core kernel (rotate_tc.cu) rotates:
-// its per-group matrices (64 KB each) then cost less than the activations
-constexpr int64_t kRotateTcMinTokens = 128;
+// above 16 tokens the tensor-core kernel (rotate_tc.cu) rotates: measured
+// faster from 17 tokens on (3.0 against 3.6 us at 17 tokens, hidden 4096, K = 8)
+constexpr int64_t kRotateTcMinTokens = 17;
 
 template <int QW, bool PF>
 cudaError_t launch_quad(const RotDev& r, const void* X, void* Xr, int64_t T, int warps, cudaStream_t s,
@@ -369,30 +269,10 @@ cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64
                  : launch_quad<1, false>(r, X, Xr, T, warps, s, lane_major ? 1 : 0);
 }
 
-template <int TT>
-static cudaError_t launch_rotate_t(const RotDev& r, const __half* x, __half* y, int64_t T, cudaStream_t s) {
-    const int64_t tasks = ((T + TT - 1) / TT) * r.G;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)((tasks + 3) / 4), 1, 1);
-    cfg.blockDim = dim3(128, 1, 1);
-    cfg.stream = s;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr.val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, rotate_kernel<TT>, x, y, T, (int)r.in, r.G, r.K, (const uint8_t*)r.rotx,
-                              (const float*)r.inv_alpha);
-}
-
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    const __half* x = static_cast<const __half*>(X);
-    __half* y = static_cast<__half*>(Xr);
-    if (T <= 16) return launch_rotate_decode(r, X, Xr, T, s);
-    if (T >= kRotateTcMinTokens) return launch_rotate_tc(r, X, Xr, T, s);
-    const cudaError_t e = launch_rotate_t<8>(r, x, y, T, s);
-    return e != cudaSuccess ? e : cudaGetLastError();
+    if (T < kRotateTcMinTokens) return launch_rotate_decode(r, X, Xr, T, s);
+    return launch_rotate_tc(r, X, Xr, T, s);
 }
 
 }  // namespace paro

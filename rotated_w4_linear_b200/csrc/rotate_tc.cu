@@ -246,7 +246,7 @@ rotate_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
 namespace {
 
-constexpr int kTcStages = 4;
+constexpr int kTcStages = 5;
 
 template <int S>
 constexpr size_t tc_smem() {

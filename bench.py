@@ -62,8 +62,8 @@ def call_bytes(T, n_in, n_out):
 # one ncu capture at 16 tokens of the decode kernel built from the gemv.cu
 # whose SHA-256 prefix is GEMV_TRAFFIC_SOURCE; reported only while gemv.cu is
 # that file (any change to it nulls the figure until it is captured again).
-GEMV_TRAFFIC_PER_LAUNCH_T16 = (13238528 + 8886272 + 61180416 + 30999040) / 4
-GEMV_TRAFFIC_SOURCE = "unset"
+GEMV_TRAFFIC_PER_LAUNCH_T16 = (13239040 + 8883968 + 61178880 + 30999040) / 4
+GEMV_TRAFFIC_SOURCE = "e96d84dec74edc6e"
 
 
 def gemv_source_sha() -> str:
@@ -190,9 +190,14 @@ def emit(line, rank):
 
 
 # --------------------------------------------------------------------------- oracle baseline
-def cpu_baseline(tokens: int, budget_s: float = 12.0):
+def cpu_baseline(tokens: int, budget_s: float = 12.0, torch=None, B=None):
     """The CPU fp64 oracle as it stands, on a bounded sample: whole projections
-    of layer 0 (every output row), one after another until ~budget_s."""
+    of one layer (every output row), one after another until ~budget_s.
+    With torch and the binding given, the four projections of that layer
+    also run through paro_linear on the GPU and are compared with the
+    oracle's outputs: the literal max |dY| beside the 1e-2 bar and the format
+    floor (the ideal fp16 pipeline's own max error), and the Frobenius error.
+    Returns (cpu_baseline, parity or None)."""
     from oracle import paro_oracle as O
     try:
         from threadpoolctl import threadpool_info
@@ -200,22 +205,40 @@ def cpu_baseline(tokens: int, budget_s: float = 12.0):
     except Exception:
         cores = 1
     done_bytes, t_total, n_calls, names = 0, 0.0, 0, []
+    par = {"max_abs_dY": 0.0, "format_floor": 0.0, "rel_fro": 0.0, "max_abs_Y": 0.0}
     for i, (name, n_in, n_out) in enumerate(PROJ * 16):
         seed = synth.layer_seed(2, i % len(PROJ))
         pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
         q, s, z = synth.w4_codes(n_out, n_in, seed)
         x = synth.activations(tokens, n_in, seed)
         t0 = time.perf_counter()
-        O.linear(x, pairs, theta, alpha, q, s, z)
+        y_ref = O.linear(x, pairs, theta, alpha, q, s, z)
         t_total += time.perf_counter() - t0
         done_bytes += call_bytes(tokens, n_in, n_out)
         n_calls += 1
         names.append(name)
+        if B is not None and i < len(PROJ):
+            rot = B.paro_rot_create(pairs, theta, alpha)
+            qw, sp, zp = B.paro_pack_weights(torch.from_numpy(q), torch.from_numpy(s), torch.from_numpy(z))
+            y = B.paro_linear(rot, torch.from_numpy(x).cuda(), qw, sp, zp, n_out).cpu().numpy().astype(np.float64)
+            rot.close()
+            floor = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z).astype(np.float64)
+            rel, mx = O.output_errors(y, y_ref)
+            par["max_abs_dY"] = max(par["max_abs_dY"], mx)
+            par["rel_fro"] = max(par["rel_fro"], rel)
+            par["format_floor"] = max(par["format_floor"], float(np.max(np.abs(floor - y_ref))))
+            par["max_abs_Y"] = max(par["max_abs_Y"], float(np.max(np.abs(y_ref))))
         if t_total > budget_s:
             break
-    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
+    base = {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
             "sample": f"{n_calls} projection calls ({'+'.join(names)}) of one layer, every output row, "
                       f"{tokens} tokens, fp64 numpy ({t_total:.1f} s)"}
+    if B is None:
+        return base, None
+    par.update({"bar_abs": 1e-2, "bar_rel": 2e-3,
+                "sample": f"the four projections of one {'-'.join(n for n, _, _ in PROJ)} layer at {tokens} tokens, "
+                          "every output, GPU paro_linear against the fp64 oracle (max over the four)"})
+    return base, par
 
 
 def run_reference(args, rank: int, world: int):
@@ -324,9 +347,10 @@ def bench_rotate(args, torch, B, local):
 def prefill_result(torch, B, local, T, steps, warmup, model):
     """One decoder layer's projections (`model` shapes) at T tokens: rotation +
     tensor-core GEMM per projection, replayed as a CUDA graph. Reports the
-    GEMM FLOP rate (2 T in out per projection) against the measured dense
-    16-bit tensor peak, and the rotation overhead against the same GEMMs on
-    unrotated inputs (theta = 0, alpha = 1: no rotation launch)."""
+    layer's FLOP rate (2 T in out per projection; the time includes the
+    rotation launches) against the measured dense 16-bit tensor peak, the
+    rotation overhead against the same GEMMs on unrotated inputs (theta = 0,
+    alpha = 1: no rotation launch), and the rotations alone."""
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     calls = []
@@ -347,28 +371,33 @@ def prefill_result(torch, B, local, T, steps, warmup, model):
             B.paro_linear(p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
                           Y=p["y"], ws=p["ws"])
 
-    step(); step(False)
+    def rotations():
+        for p in calls:
+            B.paro_rotate(p["rot"], p["x"], p["ws"][: p["x"].numel() * 2].view(torch.float16).view(p["x"].shape))
+
+    step(); step(False); rotations()
     torch.cuda.synchronize()
     graphs = {}
-    for rot in (True, False):
+    for key, fn in (("rotated", lambda: step(True)), ("unrotated", lambda: step(False)), ("rotation", rotations)):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step(rot)
-        graphs[rot] = g
+            fn()
+        graphs[key] = g
     for _ in range(warmup):
-        graphs[True].replay(); graphs[False].replay()
+        for g in graphs.values():
+            g.replay()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     times = {}
     with ClockSampler(local) as clk:
-        for rot in (True, False):
+        for key, g in graphs.items():
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for _ in range(steps):
-                graphs[rot].replay()
+                g.replay()
             e1.record(stream)
             torch.cuda.synchronize()
-            times[rot] = e0.elapsed_time(e1) / 1e3 / steps
+            times[key] = e0.elapsed_time(e1) / 1e3 / steps
     flops = sum(2.0 * T * p["n_in"] * p["n_out"] for p in calls)
     _, _, kind = peaks()
     try:
@@ -376,16 +405,21 @@ def prefill_result(torch, B, local, T, steps, warmup, model):
             tc_peak = float(json.load(f)["bf16_tflops_sustained"])
     except Exception:
         tc_peak = 1400.0
-    tf = flops / times[False] / 1e12
+    tf = flops / times["rotated"] / 1e12
     shapes = ", ".join(f"{n} {i}x{o}" for n, i, o in MODELS[model])
     res = {"workload": f"prefill {model} decoder-layer projections ({shapes}), {T} tokens, K={K_LAYERS}",
-           "ms_per_layer": 1e3 * times[True], "ms_per_layer_unrotated": 1e3 * times[False],
-           "TFLOP/s": flops / times[True] / 1e12, "TFLOP/s_gemm_only": tf,
-           "rotation_overhead": times[True] / times[False] - 1.0,
+           "ms_per_layer": 1e3 * times["rotated"], "ms_per_layer_unrotated": 1e3 * times["unrotated"],
+           "ms_rotation_alone": 1e3 * times["rotation"],
+           "TFLOP/s": tf, "TFLOP/s_unrotated_control": flops / times["unrotated"] / 1e12,
+           "rotation_overhead": times["rotated"] / times["unrotated"] - 1.0,
+           "rotation_share": times["rotation"] / times["rotated"],
            "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak, "unit": "TFLOP/s",
-                        "frac": tf / tc_peak, "traffic": None, "kernel": "gemm_w4_kernel (tcgen05)",
+                        "frac": tf / tc_peak, "traffic": None,
+                        "kernel": "gemm_w4_kernel (tcgen05), timed with its rotation launches (the whole layer)",
                         "flops_per_layer": flops,
                         "peak_source": f"{kind} bf16_tflops_sustained (fp16 and bf16 share the dense tensor rate)"},
+           "note": "the unrotated control reads X from HBM; the rotated layer's GEMM reads X' that the rotation "
+                   "just wrote, partly from L2, so the overhead can come out below zero",
            "l2": "inputs larger than L2", "clocks": clk.summary()}
     del graphs
     for p in calls:
@@ -620,7 +654,7 @@ def main():
         line["prefill"] = prefill_result(torch, B, local, 8192, xs, 3, args.model)
         torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(T)
+        line["cpu_baseline"], line["parity"] = cpu_baseline(T, torch=torch, B=B)
     emit(line, rank)
     if dist:
         dist.barrier()

@@ -57,13 +57,16 @@ typedef struct paro_rot paro_rot;
 
 /* Validate and prepare the scaled pairwise rotation T of one layer and upload
  * it to the current device (setup; allocates device memory; synchronous).
- *   in_features      multiple of `group`
- *   group            channels per quantisation group; only 128 is supported
+ *   in_features      multiple of 128
+ *   group            channels per quantisation group: 128 or 64 (256 is not
+ *                    supported: PARO_ERR_UNSUPPORTED)
  *   K                number of rotation layers, 0..16 (K = 0: T = diag(alpha))
  *   pairs_per_group  P, 1..group/2 active pairs per (layer, group)
  *   pairs_host       int16 [K][in/group][P][2], group-local channel indices
  *                    (0..group-1); (i, j) order as in the 2x2 matrix above.
  *                    Within one (layer, group) no channel may appear twice.
+ *                    (Groups of 64 are held as pairs of groups in 128-channel
+ *                    tables; a pair still never leaves its 64-channel group.)
  *   theta_host       float [K][in/group][P], radians
  *   alpha_host       float [in_features], finite and non-zero
  * Paper: ICLR 2026 notes, "key design" (Givens decomposition, independent
@@ -87,6 +90,13 @@ paro_status paro_rotate(const paro_rot* rot, const void* X_dev, void* Xr_dev,
 paro_status paro_pack_size(int64_t in_features, int64_t out_features,
                            size_t* qweight_bytes, size_t* scales_bytes, size_t* zeros_bytes);
 
+/* The same for a quantisation group of `group` channels (128 or 64; the
+ * format above is group 128): one scale word and one zero byte per group of
+ * each 16-row block's row pairs. Paper: the group size as a speed/accuracy
+ * knob (CSDN article, section 5.2). */
+paro_status paro_pack_size_ex(int64_t in_features, int64_t out_features, int group,
+                              size_t* qweight_bytes, size_t* scales_bytes, size_t* zeros_bytes);
+
 /* Pack logical W4G128 tensors into the device weight format read by
  * paro_linear (the int4 layout of the weight stream; one 16x16 tile is one
  * 32-bit word per lane of a warp, nibbles ordered for a two-instruction
@@ -106,6 +116,13 @@ paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t
                               void* qweight_dev, void* scales_dev, void* zeros_dev,
                               paro_stream stream);
 
+/* paro_pack_weights for a quantisation group of `group` channels (128 or 64):
+ * s and z are [out][in/group]; sizes from paro_pack_size_ex. */
+paro_status paro_pack_weights_ex(const uint8_t* q, const uint16_t* s, const uint8_t* z,
+                                 int64_t in_features, int64_t out_features, int group,
+                                 void* qweight_dev, void* scales_dev, void* zeros_dev,
+                                 paro_stream stream);
+
 /* Expand the device weight format back to w_hat = fp16((q - z) * s),
  * fp16 [out][in] (the dequantisation used inside paro_linear; exact product,
  * one rounding). */
@@ -113,11 +130,17 @@ paro_status paro_dequant(const void* qweight_dev, const void* scales_dev, const 
                          int64_t in_features, int64_t out_features, void* W_dev,
                          paro_stream stream);
 
+/* paro_dequant for the format of paro_pack_weights_ex with `group` (128 or 64). */
+paro_status paro_dequant_ex(const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
+                            int64_t in_features, int64_t out_features, int group, void* W_dev,
+                            paro_stream stream);
+
 /* Offline converter: W' = T W along the input axis (fp64), then asymmetric
- * RTN per 128-input group: s = fp16((max-min)/15) floored at 2^-14,
+ * RTN per input group of the handle's group size (128 or 64):
+ * s = fp16((max-min)/15) floored at 2^-14,
  * z = clamp(rint(-min/s), 0, 15), q = clamp(rint(w/s) + z, 0, 15).
  *   W_dev  fp16 [out][in] (PyTorch orientation); outputs q_dev uint8 [out][in],
- *   s_dev fp16 [out][in/128], z_dev uint8 [out][in/128].
+ *   s_dev fp16 [out][in/group], z_dev uint8 [out][in/group].
  * Paper: T W in the final-transform equation (paper notes, "key design");
  * the RTN rule is this library's reading of W4G128. */
 paro_status paro_quantize_weights(const paro_rot* rot, const void* W_dev, int64_t out_features,
@@ -163,6 +186,38 @@ paro_status paro_linear_bias(const paro_rot* rot, const void* X_dev,
                              int64_t out_features, void* workspace_dev, size_t workspace_bytes,
                              paro_stream stream);
 
+/* The general form of the layer: paro_linear_bias with weights quantised in
+ * groups of `group` channels (128 or 64, packed by paro_pack_weights_ex).
+ * A rotation handle, if given, must have been prepared with the same group
+ * (else PARO_ERR_ARG). paro_linear and paro_linear_bias are this call with
+ * group 128. Paper: CSDN article, section 2.1 (Y = (X T^-1)(T W) + b) and
+ * section 5.2 (group size). */
+paro_status paro_linear_ex(const paro_rot* rot, const void* X_dev,
+                           const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
+                           const void* bias_dev, int group, void* Y_dev, int64_t tokens, int64_t in_features,
+                           int64_t out_features, void* workspace_dev, size_t workspace_bytes,
+                           paro_stream stream);
+
+/* Row-parallel use (several GPUs each holding a slice of the input channels,
+ * cut on 128-channel boundaries): the group-diagonal T lets every rank
+ * rotate only its own channels (paper notes, "independent rotation"), so a
+ * rank's share of Y is (X_r T_r^-1) w_hat_r^T over its slice. This call
+ * writes that share as unrounded fp32 sums, Yf_dev fp32 [tokens][out]
+ * (16-byte aligned), without a bias; the ranks add their shares (an
+ * all-reduce) and paro_finalize rounds once. The rotation handle, the
+ * weights and X_dev are the rank's slice (in_features = the slice's width).
+ * Other arguments as paro_linear_ex. */
+paro_status paro_linear_partial(const paro_rot* rot, const void* X_dev,
+                                const void* qweight_dev, const void* scales_dev, const void* zeros_dev, int group,
+                                float* Yf_dev, int64_t tokens, int64_t in_features, int64_t out_features,
+                                void* workspace_dev, size_t workspace_bytes, paro_stream stream);
+
+/* Y_dev fp16 [tokens][out] = fp16(Yf_dev + bias) with one rounding; bias_dev
+ * fp16 [out] or NULL. The last step of a row-parallel layer (no counterpart
+ * in the paper beyond Y = XW + b, CSDN article, section 2.1). */
+paro_status paro_finalize(const float* Yf_dev, const void* bias_dev, void* Y_dev, int64_t tokens,
+                          int64_t out_features, paro_stream stream);
+
 /* paro_linear for decode batches (tokens <= 16) that allocates nothing and
  * takes no workspace: for callers that cannot allocate device memory, such
  * as a serving engine that hands all device memory to its own pool at start-
@@ -177,7 +232,7 @@ paro_status paro_linear_bias(const paro_rot* rot, const void* X_dev,
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) once for that device; make that first call before
  * any stream capture. Arguments are those of paro_linear without the
- * workspace; the caller still owns X, the weights and Y. */
+ * workspace (group-128 weights); the caller still owns X, the weights and Y. */
 paro_status paro_linear_noalloc(const paro_rot* rot, const void* X_dev,
                                 const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
                                 void* Y_dev, int64_t tokens, int64_t in_features, int64_t out_features,

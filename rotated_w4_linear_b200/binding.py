@@ -36,6 +36,12 @@ _SIGS = {
     "paro_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
     "paro_linear_bias": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
     "paro_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
+    "paro_pack_size_ex": [_i64, _i64, _int, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
+    "paro_pack_weights_ex": [_vp, _vp, _vp, _i64, _i64, _int, _vp, _vp, _vp, _vp],
+    "paro_dequant_ex": [_vp, _vp, _vp, _i64, _i64, _int, _vp, _vp],
+    "paro_linear_ex": [_vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
+    "paro_linear_partial": [_vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64, _vp, _sz, _vp],
+    "paro_finalize": [_vp, _vp, _vp, _i64, _i64, _vp],
     "paro_rotate_once": [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _int, _int, _int, _vp],
     "paro_linear_once": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp],
     "paro_fault_status": [ctypes.POINTER(_int), _int],
@@ -105,7 +111,7 @@ class Rotation:
         K = int(pairs.shape[0]) if pairs.ndim == 4 else 0
         P = int(pairs.shape[2]) if K else 0
         self.in_features = int(alpha.shape[0])
-        self.K, self.P = K, P
+        self.K, self.P, self.group = K, P, int(group)
         h = _vp()
         _check("paro_rot_create", lib().paro_rot_create(
             ctypes.byref(h), self.in_features, group, K, P,
@@ -150,9 +156,14 @@ def paro_check_wait_timeout(limit_us: int = 1000, stream=None) -> None:
     _check("paro_check_wait_timeout", lib().paro_check_wait_timeout(int(limit_us), _stream(stream)))
 
 
-def paro_pack_size(in_features: int, out_features: int):
+def paro_pack_size(in_features: int, out_features: int, group: int = 128):
     q, s, z = _sz(), _sz(), _sz()
-    _check("paro_pack_size", lib().paro_pack_size(in_features, out_features, ctypes.byref(q), ctypes.byref(s), ctypes.byref(z)))
+    if group == 128:
+        _check("paro_pack_size", lib().paro_pack_size(in_features, out_features, ctypes.byref(q), ctypes.byref(s),
+                                                      ctypes.byref(z)))
+    else:
+        _check("paro_pack_size_ex", lib().paro_pack_size_ex(in_features, out_features, group, ctypes.byref(q),
+                                                            ctypes.byref(s), ctypes.byref(z)))
     return q.value, s.value, z.value
 
 
@@ -163,34 +174,37 @@ def _any(t, dtype, name) -> int:
     return t.data_ptr()
 
 
-def paro_pack_weights(q: torch.Tensor, s: torch.Tensor, z: torch.Tensor, stream=None, device=None):
-    """Logical (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]), on the
-    device or on the host -> device format (qweight, scales, zeros) as uint8
-    tensors on `device` (default: q's device, else the current one)."""
+def paro_pack_weights(q: torch.Tensor, s: torch.Tensor, z: torch.Tensor, stream=None, device=None,
+                      group: int = 128):
+    """Logical (q uint8 [out][in], s fp16 [out][in/group], z uint8
+    [out][in/group]), on the device or on the host -> device format
+    (qweight, scales, zeros) as uint8 tensors on `device` (default: q's
+    device, else the current one)."""
     out_f, in_f = q.shape
-    qb, sb, zb = paro_pack_size(in_f, out_f)
+    qb, sb, zb = paro_pack_size(in_f, out_f, group)
     dev = device or (q.device if q.is_cuda else torch.device("cuda", torch.cuda.current_device()))
     qw = torch.empty(qb, dtype=torch.uint8, device=dev)
     sp = torch.empty(sb, dtype=torch.uint8, device=dev)
     zp = torch.empty(zb, dtype=torch.uint8, device=dev)
-    _check("paro_pack_weights", lib().paro_pack_weights(
-        _any(q, torch.uint8, "q"), _any(s, torch.float16, "s"), _any(z, torch.uint8, "z"), in_f, out_f,
+    _check("paro_pack_weights_ex", lib().paro_pack_weights_ex(
+        _any(q, torch.uint8, "q"), _any(s, torch.float16, "s"), _any(z, torch.uint8, "z"), in_f, out_f, group,
         qw.data_ptr(), sp.data_ptr(), zp.data_ptr(), _stream(stream, qw.device)))
     return qw, sp, zp
 
 
-def paro_dequant(qw, sp, zp, in_features: int, out_features: int, stream=None) -> torch.Tensor:
+def paro_dequant(qw, sp, zp, in_features: int, out_features: int, stream=None, group: int = 128) -> torch.Tensor:
     W = torch.empty((out_features, in_features), dtype=torch.float16, device=qw.device)
-    _check("paro_dequant", lib().paro_dequant(_dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"),
-                                              _dev(zp, torch.uint8, "zeros"), in_features, out_features,
-                                              W.data_ptr(), _stream(stream)))
+    _check("paro_dequant_ex", lib().paro_dequant_ex(_dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"),
+                                                    _dev(zp, torch.uint8, "zeros"), in_features, out_features, group,
+                                                    W.data_ptr(), _stream(stream)))
     return W
 
 
 def paro_quantize_weights(rot: Rotation, W: torch.Tensor, stream=None):
-    """W fp16 [out][in] -> (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]) of T W."""
+    """W fp16 [out][in] -> (q uint8 [out][in], s fp16 [out][G], z uint8 [out][G]) of T W,
+    G = in / the handle's group size."""
     out_f, in_f = W.shape
-    G = in_f // 128
+    G = in_f // rot.group
     q = torch.empty((out_f, in_f), dtype=torch.uint8, device=W.device)
     s = torch.empty((out_f, G), dtype=torch.float16, device=W.device)
     z = torch.empty((out_f, G), dtype=torch.uint8, device=W.device)
@@ -279,6 +293,57 @@ def paro_linear_once(X: torch.Tensor, pairs, theta, alpha, qw, sp, zp, out_featu
         alpha.ctypes.data, _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"),
         _dev(zp, torch.uint8, "zeros"), _dev(Y, torch.float16, "Y"), T, in_f, out_features, K, P,
         _stream(stream, X.device)))
+    return Y
+
+
+def paro_linear_ex(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_features: int, group: int = 128,
+                   bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                   ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The layer with weights quantised in groups of `group` channels (128 or 64)."""
+    T, in_f = X.shape
+    if Y is None:
+        Y = torch.empty((T, out_features), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(T, in_f, out_features, X.device)
+    b = None
+    if bias is not None:
+        if bias.numel() != out_features:
+            raise ValueError("bias must have out_features elements")
+        b = _dev(bias, torch.float16, "bias")
+    _check("paro_linear_ex", lib().paro_linear_ex(
+        rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
+        _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"), b, group,
+        _dev(Y, torch.float16, "Y"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
+        _stream(stream, X.device)))
+    return Y
+
+
+def paro_linear_partial(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_features: int, group: int = 128,
+                        Yf: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """A row-parallel rank's unrounded fp32 share of Y over its input slice."""
+    T, in_f = X.shape
+    if Yf is None:
+        Yf = torch.empty((T, out_features), dtype=torch.float32, device=X.device)
+    if ws is None:
+        ws = workspace(T, in_f, out_features, X.device)
+    _check("paro_linear_partial", lib().paro_linear_partial(
+        rot.handle if rot is not None else None, _dev(X, torch.float16, "X"),
+        _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), _dev(zp, torch.uint8, "zeros"), group,
+        _dev(Yf, torch.float32, "Yf"), T, in_f, out_features, _dev(ws, torch.uint8, "workspace"), ws.numel(),
+        _stream(stream, X.device)))
+    return Yf
+
+
+def paro_finalize(Yf: torch.Tensor, bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """fp16(Yf + bias), one rounding."""
+    T, out_f = Yf.shape
+    if Y is None:
+        Y = torch.empty((T, out_f), dtype=torch.float16, device=Yf.device)
+    b = _dev(bias, torch.float16, "bias") if bias is not None else None
+    _check("paro_finalize", lib().paro_finalize(_dev(Yf, torch.float32, "Yf"), b, _dev(Y, torch.float16, "Y"), T, out_f,
+                                                _stream(stream, Yf.device)))
     return Y
 
 

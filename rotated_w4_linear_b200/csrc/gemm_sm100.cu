@@ -49,13 +49,15 @@ __host__ __device__ constexpr uint32_t tmem_cols() {
 }
 
 struct GemmArgs {
-    int T, in, out, G, Gp, nkb, nrb;
+    int T, in, out, G, Gp, nkb, nrb;   // G: quantisation groups along in (Gp: rounded up to even)
+    int gshift;                 // 64-wide k block kb lies in group kb >> gshift (1: group 128, 0: group 64)
     int kb_per_split;           // 64-wide k blocks per CTA along grid z (even: splits start on a group)
     int nsplit;                 // CTAs along z = cluster size along z (split-k)
     const uint32_t* sp;
     const uint8_t* zp;
     const __half* bias;         // [out] fp16 or null
-    __half* Y;
+    __half* Y;                  // fp16 [T][out], or
+    float* Yf;                  // fp32 [T][out] unrounded sums (row-parallel partials) when not null
 };
 
 __device__ __forceinline__ void cluster_barrier() {
@@ -142,7 +144,7 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 const int s = i % STAGES, u = i / STAGES;
                 if (u > 0 && !mbar_wait(free0 + 8 * s, (u - 1) & 1, kFaultTmaWait, abort)) break;
                 if (*abort) break;
-                const int kb = kblock(i), gi = kb >> 1;
+                const int kb = kblock(i), gi = kb >> a.gshift;
                 mbar_arrive_expect_tx(full0 + 8 * s, kBStage + kWStage + kSStage + kZStage);
                 tma_load_2d(smem_addr(sB + s * kBStage), &tm_x, kb * 64, n0, full0 + 8 * s);
                 tma_load_2d(smem_addr(sW + s * kWStage), &tm_w, kb * 128, rb0, full0 + 8 * s);
@@ -185,7 +187,7 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int g = lane >> 2;
         for (int i = dg; i < nk; i += DQG) {
             const int s = i % STAGES, u = i / STAGES;
-            const int gi = kblock(i) >> 1;
+            const int gi = kblock(i) >> a.gshift;
             // the tensor-memory stores below are warp-collective: the whole
             // warp goes on only if every lane saw the stage arrive
             if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8 * s, u & 1, kFaultDequantWait, abort) && !*abort))
@@ -238,7 +240,10 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int t = n0 + c0 + j;
-                        if (t < a.T) a.Y[(size_t)t * a.out + row] = __float2half_rn(__uint_as_float(r[j]) + b);
+                        if (t < a.T) {
+                            if (a.Yf) a.Yf[(size_t)t * a.out + row] = __uint_as_float(r[j]) + b;
+                            else a.Y[(size_t)t * a.out + row] = __float2half_rn(__uint_as_float(r[j]) + b);
+                        }
                     }
                 }
             }
@@ -258,8 +263,11 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const int row = rb0 * 16 + rl;
             float sum = 0.f;
             for (int x = 0; x < a.nsplit; ++x) sum += ld_cluster_f32(red_addr + (uint32_t)(t * kRedStride + rl) * 4u, (uint32_t)x);
-            if (t < a.T && row < a.out)
-                a.Y[(size_t)t * a.out + row] = __float2half_rn(sum + (a.bias ? __half2float(a.bias[row]) : 0.f));
+            if (t < a.T && row < a.out) {
+                const float v = sum + (a.bias ? __half2float(a.bias[row]) : 0.f);
+                if (a.Yf) a.Yf[(size_t)t * a.out + row] = v;
+                else a.Y[(size_t)t * a.out + row] = __float2half_rn(v);
+            }
         }
         cluster_barrier();                                // partial tiles stay alive until all reads are done
     } else {
@@ -352,6 +360,7 @@ cudaError_t launch_cfg(const CUtensorMap* tm, const GemmArgs& a, int mt, int nt,
 // tm[1]: packed int4 codes as uint32 [out/16][in/64 * 128], box one k block x 8 row blocks
 // tm[2]: scales uint32 [out/16][G * 8], box one group x 8 row blocks
 // tm[3]: zeros uint8 [out/16][Gp * 8], box two groups x 8 row blocks
+// (G quantisation groups of 128 or 64 channels)
 bool encode_maps(const void* Xr, const void* qw, const void* sp, const void* zp, int64_t T, int BN,
                  const GemmArgs& a, CUtensorMap* tm) {
     return encode_tma_2d(&tm[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xr, (uint64_t)a.in, (uint64_t)T, (uint64_t)a.in * 2,
@@ -364,12 +373,14 @@ bool encode_maps(const void* Xr, const void* qw, const void* sp, const void* zp,
                      (uint64_t)a.Gp * 8, 16u, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-GemmArgs make_args(int64_t T, int64_t in, int64_t out, const void* scp, const void* zp, const void* bias, void* Y) {
+GemmArgs make_args(int64_t T, int64_t in, int64_t out, int group, const void* scp, const void* zp, const void* bias,
+                   void* Y, bool y_fp32) {
     GemmArgs a{};
     a.T = (int)T;
     a.in = (int)in;
     a.out = (int)out;
-    a.G = (int)(in / 128);
+    a.G = (int)(in / group);
+    a.gshift = group == 64 ? 0 : 1;
     a.Gp = a.G + (a.G & 1);
     a.nkb = (int)(in / 64);
     a.nrb = (int)(out / 16);
@@ -378,17 +389,19 @@ GemmArgs make_args(int64_t T, int64_t in, int64_t out, const void* scp, const vo
     a.sp = static_cast<const uint32_t*>(scp);
     a.zp = static_cast<const uint8_t*>(zp);
     a.bias = static_cast<const __half*>(bias);
-    a.Y = static_cast<__half*>(Y);
+    a.Y = y_fp32 ? nullptr : static_cast<__half*>(Y);
+    a.Yf = y_fp32 ? static_cast<float*>(Y) : nullptr;
     return a;
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, const void* bias, void* Y,
-                        int64_t T, int64_t in, int64_t out, cudaStream_t s) {
+                        int64_t T, int64_t in, int64_t out, int group, cudaStream_t s, bool y_fp32) {
     if (T <= 0) return cudaSuccess;
+    if (group != 64 && group != 128) return cudaErrorInvalidValue;
     const int BN = T <= 64 ? 64 : T <= 128 ? 128 : 256;
-    GemmArgs a = make_args(T, in, out, scp, zp, bias, Y);
+    GemmArgs a = make_args(T, in, out, group, scp, zp, bias, Y, y_fp32);
     CUtensorMap tm[4];
     if (!encode_maps(Xr, qw, scp, zp, T, BN, a, tm)) return cudaErrorInvalidValue;
     const int mt = (a.nrb + 7) / 8;

@@ -50,13 +50,17 @@ namespace {
 constexpr int kWarps = 16;
 constexpr int kStages = 3;
 constexpr int kMaxSplit = 16;                             // largest cluster (k-chunks per row tile)
-constexpr int kItemGroups = 2;                            // groups per item
+constexpr int kItemGroups = 2;                            // 128-channel groups per item
 constexpr int kItemQBytes = kItemGroups * 2 * 512;        // int4 codes
-constexpr int kItemBytes = kItemQBytes + kItemGroups * 32 + 16;   // + scales + zeros
+// GS: quantisation groups per 128 channels (1: group 128, 2: group 64); an
+// item carries codes, then GS scale words x 8 per group, then GS zero bytes x 8
+template <int GS>
+constexpr int item_bytes() { return kItemQBytes + kItemGroups * GS * 32 + kItemGroups * GS * 8; }
 
 struct GemvArgs {
     const __half* Xr;     // [T][in] fp16, already rotated
-    int T, in, out, G, Gp;
+    int T, in, out, G;    // G: 128-channel groups
+    int Gq, Gqp;          // quantisation groups (scales and zeros) along in; Gqp rounded up to even
     int KC;               // groups per k-chunk (last chunk may be shorter)
     int RT;               // row blocks per CTA
     int nsplit;           // k-chunks = cluster size along x
@@ -65,7 +69,8 @@ struct GemvArgs {
     const uint32_t* sp;
     const uint8_t* zp;
     const __half* bias;   // [out] fp16 or null
-    __half* Y;
+    __half* Y;            // fp16 [T][out], or
+    float* Yf;            // fp32 [T][out] unrounded sums (row-parallel partials) when not null
     int xlm;              // X' already lane-major within 64-channel blocks
 };
 
@@ -120,42 +125,46 @@ __device__ __forceinline__ void cluster_sync_relaxed() {
 }
 
 // A lane's source pointers for the items of one row block: codes (the
-// lane's 16 bytes of each 512-byte k block), scales (lanes 0..3: 16 bytes
-// each) and zeros (lanes 30, 31: 8 bytes per group). Within a row block the
-// next group is 1 KB, 32 B and 8 B further on.
+// lane's 16 bytes of each 512-byte k block), scales (lanes 0..2 GS - 1: 16
+// bytes each) and zeros (the last 2 GS lanes: 8 bytes per quantisation
+// group). Within a row block the next 128-channel group is 1 KB, 32 GS B and
+// 8 GS B further on.
 struct ItemSrc {
     const uint4* q;
     const uint32_t* sc;
     const uint8_t* z;
 };
 
+template <int GS>
 __device__ __forceinline__ ItemSrc item_src(const GemvArgs& a, int rb, int g0, int lane) {
     const int nkb = a.in >> 6;
     ItemSrc p;
     p.q = a.qw + ((size_t)rb * nkb + 2 * g0) * 32 + lane;
-    p.sc = a.sp + ((size_t)rb * a.G + g0) * 8 + lane * 4;
-    p.z = a.zp + ((size_t)rb * a.Gp + g0) * 8;
+    p.sc = a.sp + ((size_t)rb * a.Gq + GS * g0) * 8 + lane * 4;
+    p.z = a.zp + ((size_t)rb * a.Gqp + GS * g0) * 8;
     return p;
 }
 
 // Copy one item (groups g0, g0+1 if ng == 2 of the source's row block) into
 // a ring slot; `dst` is the slot address plus this lane's 16-byte offset.
-// Slot layout: codes [2 ng][512 B], scales [ng][32 B] at kItemQBytes, zeros
-// [ng][8 B] after the scales of kItemGroups groups.
+// Slot layout: codes [2 ng][512 B], scales [GS ng][32 B] at kItemQBytes,
+// zeros [GS ng][8 B] after the scales of kItemGroups groups.
+template <int GS>
 __device__ __forceinline__ void issue_item(const ItemSrc& p, uint32_t slot, uint32_t dst, int ng, int lane) {
 #pragma unroll
     for (int kb = 0; kb < 2 * kItemGroups; ++kb) cp_async16_if(kb < 2 * ng, dst + kb * 512, p.q + kb * 32);
-    cp_async16_if(lane < 2 * ng, slot + kItemQBytes + lane * 16, p.sc);
-    // zeros: 8 bytes per group from lanes 30 and 31 (an item may start at an
-    // odd group, so the pair need not be 16-byte aligned)
-    const int zg = lane & 1;
-    cp_async8_if(lane >= 32 - kItemGroups && zg < ng, slot + kItemQBytes + kItemGroups * 32 + 8 * zg, p.z + 8 * zg);
+    cp_async16_if(lane < 2 * GS * ng, slot + kItemQBytes + lane * 16, p.sc);
+    // zeros: 8 bytes per quantisation group from the last lanes (an item may
+    // start at an odd group, so a pair need not be 16-byte aligned)
+    const int zg = lane - (32 - kItemGroups * GS);
+    cp_async8_if(zg >= 0 && zg < GS * ng, slot + kItemQBytes + kItemGroups * GS * 32 + 8 * zg, p.z + 8 * zg);
 }
 
 }  // namespace
 
-template <int NT>
+template <int NT, int GS>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) {
+    constexpr int kItemBytes = item_bytes<GS>();
     // When the next kernel on the stream may launch (it prefetches only its
     // weights, or its tables, before it waits for this grid to complete):
     // at 8 tokens or fewer right away; above that once every warp of the CTA
@@ -196,21 +205,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
     // producer cursor: position, row block and group of the next item to
     // copy and the lane's source pointers, advanced incrementally
     int p_f = f_lo, p_rb = rb_begin + rbl_lo, p_g = g_lo;
-    ItemSrc src = item_src(a, p_rb, p_g, lane);
+    ItemSrc src = item_src<GS>(a, p_rb, p_g, lane);
     auto issue_next = [&](int stage) {
         const int ng = min(min(kItemGroups, g_end - p_g), f_hi - p_f);
         const uint32_t slot = ring_w + stage * kItemBytes;
-        issue_item(src, slot, slot + lane * 16, ng, lane);
+        issue_item<GS>(src, slot, slot + lane * 16, ng, lane);
         p_f += ng;
         p_g += ng;
         if (p_g == g_end) {
             p_g = g_begin;
             ++p_rb;
-            src = item_src(a, p_rb, g_begin, lane);
+            src = item_src<GS>(a, p_rb, g_begin, lane);
         } else {
             src.q += ng * 2 * 32;
-            src.sc += ng * 8;
-            src.z += ng * 8;
+            src.sc += ng * GS * 8;
+            src.z += ng * GS * 8;
         }
     };
 
@@ -315,10 +324,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         for (int g = 0; g < kItemGroups; ++g) {
             if (g < ng) {
                 uint32_t sc0, sc1;
-                const Zero2 zc = zero_consts(slot[kItemQBytes + kItemGroups * 32 + g * 8 + gq]);
-                scale_pairs(*reinterpret_cast<const uint32_t*>(slot + kItemQBytes + g * 32 + gq * 4), sc0, sc1);
+                Zero2 zc = zero_consts(slot[kItemQBytes + kItemGroups * GS * 32 + GS * g * 8 + gq]);
+                scale_pairs(*reinterpret_cast<const uint32_t*>(slot + kItemQBytes + GS * g * 32 + gq * 4), sc0, sc1);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
+                    if (GS == 2 && h == 1) {                   // group 64: the second half has its own s, z
+                        zc = zero_consts(slot[kItemQBytes + kItemGroups * GS * 32 + (GS * g + 1) * 8 + gq]);
+                        scale_pairs(*reinterpret_cast<const uint32_t*>(slot + kItemQBytes + (GS * g + 1) * 32 + gq * 4),
+                                    sc0, sc1);
+                    }
                     const uint4 wv = *reinterpret_cast<const uint4*>(slot + (2 * g + h) * 512 + lane * 16);
                     const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
                     // B values of the block's four k tiles: two 16-byte loads per token tile
@@ -372,7 +386,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
         for (int i = threadIdx.x; i < a.T * nrows_tile; i += kWarps * 32) {
             const int t = i / nrows_tile, r = i - t * nrows_tile;
             const float b = a.bias ? __half2float(a.bias[row0 + r]) : 0.f;
-            a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * SR + r] + b);
+            if (a.Yf) a.Yf[(size_t)t * a.out + row0 + r] = red[t * SR + r] + b;
+            else a.Y[(size_t)t * a.out + row0 + r] = __float2half_rn(red[t * SR + r] + b);
         }
         return;
     }
@@ -405,8 +420,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const GemvArgs a) 
             sum.z += __half2float(a.bias[row0 + r + 2]);
             sum.w += __half2float(a.bias[row0 + r + 3]);
         }
-        *reinterpret_cast<uint2*>(a.Y + (size_t)t * a.out + row0 + r) =
-            make_uint2(pack_half2(sum.x, sum.y), pack_half2(sum.z, sum.w));
+        if (a.Yf)
+            *reinterpret_cast<float4*>(a.Yf + (size_t)t * a.out + row0 + r) = sum;
+        else
+            *reinterpret_cast<uint2*>(a.Y + (size_t)t * a.out + row0 + r) =
+                make_uint2(pack_half2(sum.x, sum.y), pack_half2(sum.z, sum.w));
     }
     cluster_sync_relaxed();                                // tiles stay alive until every reader is done
 }
@@ -418,15 +436,15 @@ struct GemvPlan {
     size_t smem;
 };
 
-size_t gemv_smem(int NT, int KC, int RT) {
+size_t gemv_smem(int NT, int GS, int KC, int RT) {
     return (size_t)NT * 8 * (KC * 128 + 8) * 2 + (size_t)NT * 8 * (RT * 16 + 4) * 4 +
-           (size_t)kWarps * kStages * kItemBytes;
+           (size_t)kWarps * kStages * (GS == 2 ? item_bytes<2>() : item_bytes<1>());
 }
 
 // CTAs of one launch that can be resident at once: clusters of `nsplit` CTAs
 // must sit inside one GPC, so for nsplit > 1 this is the driver's count of
 // co-resident clusters times nsplit (fewer than SMs x CTAs per SM).
-template <int NT>
+template <int NT, int GS>
 int gemv_slots(int dev, int nsplit, int per_sm) {
     static std::mutex mu;
     static std::map<std::tuple<int, int, int>, int> cache;
@@ -437,7 +455,7 @@ int gemv_slots(int dev, int nsplit, int per_sm) {
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int slots = sms * per_sm;
-    if (nsplit > 1 && cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+    if (nsplit > 1 && cudaFuncSetAttribute(gemv_kernel<NT, GS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
                           cudaSuccess) {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(nsplit, 1024, 1);
@@ -451,9 +469,9 @@ int gemv_slots(int dev, int nsplit, int per_sm) {
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int nc = 0;
-        if (cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
+        if (cudaFuncSetAttribute(gemv_kernel<NT, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ==
                 cudaSuccess &&
-            cudaOccupancyMaxActiveClusters(&nc, gemv_kernel<NT>, &cfg) == cudaSuccess && nc > 0)
+            cudaOccupancyMaxActiveClusters(&nc, gemv_kernel<NT, GS>, &cfg) == cudaSuccess && nc > 0)
             slots = std::min(slots, nc * nsplit);
         cudaGetLastError();   // a refused query leaves the SM-count estimate
     }
@@ -463,7 +481,7 @@ int gemv_slots(int dev, int nsplit, int per_sm) {
 
 // Choose (k-chunk, row tile) for one shape: minimise waves x (items per warp
 // + pipeline fill), counting only CTAs that can be resident together.
-template <int NT>
+template <int NT, int GS>
 GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
     const int G = (int)(in / 128);
     const int nrb = (int)(out / 16);
@@ -479,14 +497,14 @@ GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
         const int ns = (G + KC - 1) / KC;
         if (ns != nsplit) continue;
         for (int RT = 1; RT <= std::min(nrb, 64); ++RT) {
-            const size_t smem = gemv_smem(NT, KC, RT);
+            const size_t smem = gemv_smem(NT, GS, KC, RT);
             if (smem > 200 * 1024) break;
             // one CTA of 16 warps per SM (one copy of the X' chunk per SM),
             // with room beside it for one CTA of the rotation kernel that
             // runs before this one
             if (smem + kReserved + rot_reserve > kSmemPerSm) break;
             const int per_sm = 1;
-            const int slots = gemv_slots<NT>(dev, ns, per_sm);
+            const int slots = gemv_slots<NT, GS>(dev, ns, per_sm);
             const int rowtiles = (nrb + RT - 1) / RT;
             const int ctas = ns * rowtiles;
             const int waves = (ctas + slots - 1) / slots;
@@ -514,18 +532,18 @@ GemvPlan plan_gemv(int dev, int64_t in, int64_t out, int T, int K) {
     return best;
 }
 
-template <int NT>
+template <int NT, int GS>
 GemvPlan cached_plan(int dev, int64_t in, int64_t out, int T, int K) {
     static std::mutex mu;
     static std::map<std::tuple<int, int64_t, int64_t, int, int>, GemvPlan> cache;
     std::lock_guard<std::mutex> lock(mu);
     const auto key = std::make_tuple(dev, in, out, T, K);
     auto it = cache.find(key);
-    if (it == cache.end()) it = cache.emplace(key, plan_gemv<NT>(dev, in, out, T, K)).first;
+    if (it == cache.end()) it = cache.emplace(key, plan_gemv<NT, GS>(dev, in, out, T, K)).first;
     return it->second;
 }
 
-template <int NT>
+template <int NT, int GS>
 cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, int dev, cudaStream_t s) {
     // kernel attributes, set once per device (double-checked under a lock)
     static std::atomic<bool> configured[64] = {};
@@ -535,9 +553,9 @@ cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, int dev, cudaStr
         std::lock_guard<std::mutex> lock(mu);
         if (!configured[dev].load(std::memory_order_relaxed)) {
             cudaError_t e =
-                cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+                cudaFuncSetAttribute(gemv_kernel<NT, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+                e = cudaFuncSetAttribute(gemv_kernel<NT, GS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (e != cudaSuccess) return e;
             configured[dev].store(true, std::memory_order_release);
         }
@@ -558,7 +576,7 @@ cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, int dev, cudaStr
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<NT>, a);
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, GS>, a);
 }
 
 }  // namespace
@@ -567,8 +585,11 @@ cudaError_t launch_gemv_t(const GemvArgs& a, const GemvPlan& p, int dev, cudaStr
 // null), then the decode kernel runs on it; both are programmatic dependent
 // launches, so the decode kernel's weight stream starts during the rotation.
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
-                        const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s) {
+                        const void* bias, void* Y, int64_t T, int64_t in, int64_t out, int group, void* ws,
+                        cudaStream_t s, bool y_fp32) {
     if (T <= 0) return cudaSuccess;
+    if (group != 64 && group != 128) return cudaErrorInvalidValue;
+    const bool g64 = group == 64;
     int dev = 0;
     cudaGetDevice(&dev);
     const int K = rot ? rot->K : 0;
@@ -578,14 +599,16 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
         if (e != cudaSuccess) return e;
         xr = ws;
     }
-    const GemvPlan p = (T > 8) ? cached_plan<2>(dev, in, out, (int)T, K) : cached_plan<1>(dev, in, out, (int)T, K);
+    const GemvPlan p = (T > 8) ? (g64 ? cached_plan<2, 2>(dev, in, out, (int)T, K) : cached_plan<2, 1>(dev, in, out, (int)T, K))
+                               : (g64 ? cached_plan<1, 2>(dev, in, out, (int)T, K) : cached_plan<1, 1>(dev, in, out, (int)T, K));
     GemvArgs a{};
     a.Xr = static_cast<const __half*>(xr);
     a.T = (int)T;
     a.in = (int)in;
     a.out = (int)out;
     a.G = (int)(in / 128);
-    a.Gp = a.G + (a.G & 1);
+    a.Gq = (int)(in / group);
+    a.Gqp = a.Gq + (a.Gq & 1);
     a.KC = p.KC;
     a.RT = p.RT;
     a.nsplit = p.nsplit;
@@ -594,9 +617,11 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.sp = static_cast<const uint32_t*>(scp);
     a.zp = static_cast<const uint8_t*>(zp);
     a.bias = static_cast<const __half*>(bias);
-    a.Y = static_cast<__half*>(Y);
+    a.Y = y_fp32 ? nullptr : static_cast<__half*>(Y);
+    a.Yf = y_fp32 ? static_cast<float*>(Y) : nullptr;
     a.xlm = rot ? 1 : 0;
-    cudaError_t e = (T > 8) ? launch_gemv_t<2>(a, p, dev, s) : launch_gemv_t<1>(a, p, dev, s);
+    cudaError_t e = (T > 8) ? (g64 ? launch_gemv_t<2, 2>(a, p, dev, s) : launch_gemv_t<2, 1>(a, p, dev, s))
+                            : (g64 ? launch_gemv_t<1, 2>(a, p, dev, s) : launch_gemv_t<1, 1>(a, p, dev, s));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -655,7 +680,7 @@ cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw
     void* scratch = nullptr;
     cudaError_t e = noalloc_scratch(&scratch);
     if (e != cudaSuccess) return e;
-    return launch_gemv(rot, X, qw, scp, zp, nullptr, Y, T, in, out, scratch, s);
+    return launch_gemv(rot, X, qw, scp, zp, nullptr, Y, T, in, out, 128, scratch, s);
 }
 
 }  // namespace paro

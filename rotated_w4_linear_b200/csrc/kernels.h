@@ -9,9 +9,10 @@ namespace paro {
 
 struct RotDev {
     int64_t in = 0;         // input features
-    int G = 0;              // groups of 128
+    int G = 0;              // groups of 128 (tables are built per 128 channels)
     int K = 0;              // rotation layers
-    int P = 0;              // active pairs per (layer, group)
+    int P = 0;              // active pairs per (layer, 128-channel group)
+    int group = 128;        // the layer's group size (64: two groups share each 128-channel table)
     uint8_t* rotq = nullptr;       // [K][G] quad exchange blocks (decode prologue)
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha
     uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
@@ -38,17 +39,21 @@ cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64
                                  bool lane_major = false);
 size_t rotate_decode_smem(int K, int T);
 
-cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out,
+// group: channels per quantisation group (128 or 64) of the weight format.
+cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out, int group,
                         void* qw, void* scp, void* zp, cudaStream_t s);
-cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int64_t in, int64_t out,
+cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int64_t in, int64_t out, int group,
                            void* W, cudaStream_t s);
 cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t* q, uint16_t* sc,
                             uint8_t* z, cudaStream_t s);
 
 // Decode path (tokens <= 16): the decode rotation kernel into ws (when rot
 // is not null), then the int4 decode kernel, both programmatic dependent launches.
+// group: channels per quantisation group of the weights (128 or 64).
+// y_fp32: Y is fp32 and receives the unrounded sums (row-parallel partials).
 cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const void* scp, const void* zp,
-                        const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws, cudaStream_t s);
+                        const void* bias, void* Y, int64_t T, int64_t in, int64_t out, int group, void* ws,
+                        cudaStream_t s, bool y_fp32 = false);
 
 // Decode with the X' scratch in a static device array (no allocation anywhere).
 size_t noalloc_scratch_bytes();
@@ -57,8 +62,13 @@ cudaError_t launch_gemv_noalloc(const RotDev* rot, const void* X, const void* qw
 
 // Prefill (tokens > 16): tcgen05 GEMM on X' (already rotated, in global memory),
 // launched as a programmatic dependent of the rotation kernel.
+// group: channels per quantisation group of the weights (128 or 64).
 cudaError_t launch_gemm(const void* Xr, const void* qw, const void* scp, const void* zp, const void* bias, void* Y,
-                        int64_t T, int64_t in, int64_t out, cudaStream_t s);
+                        int64_t T, int64_t in, int64_t out, int group, cudaStream_t s, bool y_fp32 = false);
+
+// Y16 = fp16(Yf + bias) (bias fp16 [out] or null): the last step of a
+// row-parallel layer after the partial sums were added across ranks.
+cudaError_t launch_finalize(const float* Yf, const void* bias, void* Y, int64_t T, int64_t out, cudaStream_t s);
 
 // A kernel whose bounded wait runs out on purpose after limit_ns (fault code 6).
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t s);

@@ -50,12 +50,12 @@ __global__ void pack_meta_kernel(const uint16_t* __restrict__ s, const uint8_t* 
     if ((G & 1) && gi == G - 1) zp[(rb * Gp + G) * 8 + g] = 0;   // padding group
 }
 
-cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out,
+cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, int64_t in, int64_t out, int group,
                         void* qw, void* scp, void* zp, cudaStream_t s) {
     const int64_t nwords = in * out / 8;
     if (nwords > 0)
         pack_q_kernel<<<(unsigned)((nwords + 255) / 256), 256, 0, s>>>(q, static_cast<uint32_t*>(qw), (int)in, nwords);
-    const int G = (int)(in / 128);
+    const int G = (int)(in / group);
     const int64_t nm = (out / 16) * G * 8;
     if (nm > 0)
         pack_meta_kernel<<<(unsigned)((nm + 255) / 256), 256, 0, s>>>(sc, z, static_cast<uint32_t*>(scp),
@@ -68,17 +68,18 @@ cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, 
 // conversion the GEMV and GEMM kernels use.
 // ---------------------------------------------------------------------------
 __global__ void dequant_kernel(const uint32_t* __restrict__ qw, const uint32_t* __restrict__ sp,
-                               const uint8_t* __restrict__ zp, __half* __restrict__ W, int in, int64_t nwords) {
+                               const uint8_t* __restrict__ zp, __half* __restrict__ W, int in, int gshift,
+                               int64_t nwords) {
     const int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (w >= nwords) return;
-    const int nkb = in / 64, G = in / 128;
+    const int nkb = in / 64, G = nkb >> gshift;               // quantisation groups of 64 << gshift channels
     const int j = (int)(w & 3);
     const int lane = (int)((w >> 2) & 31);
     const int64_t blk = w >> 7;
     const int kb = (int)(blk % nkb);
     const int64_t rb = blk / nkb;
     const int g = lane >> 2, qd = lane & 3;
-    const int gi = kb >> 1;
+    const int gi = kb >> gshift;
     const int64_t mi = (rb * G + gi) * 8 + g;
     const int Gp = G + (G & 1);
     uint32_t sc0, sc1, h[4];
@@ -91,18 +92,19 @@ __global__ void dequant_kernel(const uint32_t* __restrict__ qw, const uint32_t* 
     *reinterpret_cast<uint2*>(r0 + 8 * (int64_t)in) = make_uint2(h[2], h[3]);
 }
 
-cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int64_t in, int64_t out,
+cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int64_t in, int64_t out, int group,
                            void* W, cudaStream_t s) {
     const int64_t nwords = in * out / 8;
     if (nwords > 0)
         dequant_kernel<<<(unsigned)((nwords + 255) / 256), 256, 0, s>>>(
             static_cast<const uint32_t*>(qw), static_cast<const uint32_t*>(scp), static_cast<const uint8_t*>(zp),
-            static_cast<__half*>(W), (int)in, nwords);
+            static_cast<__half*>(W), (int)in, group == 64 ? 0 : 1, nwords);
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Offline converter: one warp per (output row, 128-input group), fp64.
+// Offline converter: one warp per (output row, 128-input group), fp64
+// (groups of 64: each half warp quantises one).
 // W'[o, c] = (T W[o, :])_c: multiply by alpha, then layers t = 1..K with
 // each channel becoming a * v + b * v_partner (two rounded products and one
 // rounded sum, no fused multiply-add, the order a plain fp64 evaluation of the
@@ -111,7 +113,8 @@ cudaError_t launch_dequant(const void* qw, const void* scp, const void* zp, int6
 constexpr int kRot64BlockBytes = 128 + 128 * 16;
 
 __global__ void __launch_bounds__(128) quantize_kernel(const __half* __restrict__ W, int in, int G, int K,
-                                                       int64_t out, const uint8_t* __restrict__ rotp64,
+                                                       int half_groups, int64_t out,
+                                                       const uint8_t* __restrict__ rotp64,
                                                        const double* __restrict__ alpha64,
                                                        uint8_t* __restrict__ q, uint16_t* __restrict__ sc,
                                                        uint8_t* __restrict__ z) {
@@ -144,10 +147,13 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __half* __restrict_
             v[r] = __dadd_rn(__dmul_rn(ab.x, v[r]), __dmul_rn(ab.y, p[r]));
         }
     }
+    // min and max over the quantisation group: the whole warp (128
+    // channels), or each half warp (64 channels) when half_groups is set
     double mn = fmin(fmin(v[0], v[1]), fmin(v[2], v[3]));
     double mx = fmax(fmax(v[0], v[1]), fmax(v[2], v[3]));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
+        if (half_groups && off == 16) continue;
         mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
         mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
@@ -166,7 +172,13 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __half* __restrict_
         packed |= (uint32_t)qd << (8 * r);
     }
     *reinterpret_cast<uint32_t*>(q + o * in + c0) = packed;
-    if (lane == 0) {
+    if (half_groups) {                                     // groups of 64: two per warp
+        if ((lane & 15) == 0) {
+            const int64_t gq = o * (2 * G) + 2 * gi + (lane >> 4);
+            sc[gq] = __half_as_ushort(s16);
+            z[gq] = (uint8_t)zd;
+        }
+    } else if (lane == 0) {
         sc[o * G + gi] = __half_as_ushort(s16);
         z[o * G + gi] = (uint8_t)zd;
     }
@@ -177,7 +189,8 @@ cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t
     const int64_t tasks = out * r.G;
     if (tasks > 0)
         quantize_kernel<<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(static_cast<const __half*>(W), (int)r.in, r.G,
-                                                                    r.K, out, r.rotp64, r.alpha64, q, sc, z);
+                                                                    r.K, r.group == 64 ? 1 : 0, out, r.rotp64,
+                                                                    r.alpha64, q, sc, z);
     return cudaGetLastError();
 }
 

@@ -124,6 +124,7 @@ paro_status paro_linear_noalloc(const paro_rot* r, const void* X, const void* qw
         return fail(PARO_ERR_ARG, "tokens x in_features x 2 = %zu bytes exceeds the %zu-byte static scratch",
                     (size_t)T * (size_t)in * 2, paro::noalloc_scratch_bytes());
     if (r && r->dev.in != in) return fail(PARO_ERR_ARG, "rotation prepared for in=%lld, layer has in=%lld", (long long)r->dev.in, (long long)in);
+    if (r && r->dev.group != 128) return fail(PARO_ERR_UNSUPPORTED, "this entry point serves group 128");
     if (!X || !qw || !sp || !zp || !Y) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(X) || !aligned16(qw) || !aligned16(sp) || !aligned16(zp) || !aligned16(Y))
         return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
@@ -151,12 +152,15 @@ paro_status paro_check_wait_timeout(uint32_t limit_us, paro_stream stream) {
     return e == cudaSuccess ? PARO_OK : cuda_fail(e, "wait self-test launch");
 }
 
-paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P, const int16_t* pairs,
-                            const float* theta, const float* alpha) {
-    g_err[0] = 0;
-    if (!out) return fail(PARO_ERR_ARG, "out is null");
-    *out = nullptr;
-    if (group != 128) return fail(PARO_ERR_UNSUPPORTED, "group=%d: only 128 is supported", group);
+}  // extern "C"
+
+namespace {
+
+// The handle for 128-channel groups (group = 128 as the caller sees it, or
+// pairs of 64-channel groups folded into 128-channel tables).
+paro_status rot_create_128(paro_rot** out, int64_t in, int K, int P, const int16_t* pairs, const float* theta,
+                           const float* alpha) {
+    const int group = 128;
     if (in <= 0 || in % group) return fail(PARO_ERR_ARG, "in_features=%lld must be a positive multiple of %d", (long long)in, group);
     if (in > (1LL << 20)) return fail(PARO_ERR_UNSUPPORTED, "in_features too large");
     if (K < 0 || K > 16) return fail(PARO_ERR_ARG, "K=%d must be in 0..16", K);
@@ -310,6 +314,47 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     return PARO_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P, const int16_t* pairs,
+                            const float* theta, const float* alpha) {
+    g_err[0] = 0;
+    if (!out) return fail(PARO_ERR_ARG, "out is null");
+    *out = nullptr;
+    if (group != 128 && group != 64)
+        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
+    if (in <= 0 || in % 128)
+        return fail(PARO_ERR_ARG, "in_features=%lld must be a positive multiple of 128", (long long)in);
+    if (K < 0 || K > 16) return fail(PARO_ERR_ARG, "K=%d must be in 0..16", K);
+    if (K > 0 && (P < 1 || P > group / 2)) return fail(PARO_ERR_ARG, "pairs_per_group=%d must be in 1..%d", P, group / 2);
+    if (K > 0 && (!pairs || !theta)) return fail(PARO_ERR_ARG, "pairs/theta is null");
+    if (group == 128) return rot_create_128(out, in, K, P, pairs, theta, alpha);
+    // groups of 64: the pairs of 64-channel groups 2h and 2h + 1 (indices
+    // 0..63 each) form the 128-channel table h, the second group's indices
+    // moved up by 64; a pair cannot leave its 64-channel group
+    const int64_t G64 = in / 64, G = in / 128;
+    std::vector<int16_t> p128((size_t)K * G * 2 * P * 2);
+    std::vector<float> t128((size_t)K * G * 2 * P);
+    for (int t = 0; t < K; ++t)
+        for (int64_t g = 0; g < G64; ++g)
+            for (int p = 0; p < P; ++p) {
+                const size_t src = ((size_t)t * G64 + g) * P + p;
+                const int i = pairs[2 * src], j = pairs[2 * src + 1];
+                if (i < 0 || i >= 64 || j < 0 || j >= 64)
+                    return fail(PARO_ERR_ARG, "pair (%d,%d) of layer %d group %lld leaves its 64-channel group", i, j,
+                                t, (long long)g);
+                const size_t dst = ((size_t)t * G + g / 2) * (2 * P) + (size_t)(g & 1) * P + p;
+                p128[2 * dst] = (int16_t)(i + 64 * (g & 1));
+                p128[2 * dst + 1] = (int16_t)(j + 64 * (g & 1));
+                t128[dst] = theta[src];
+            }
+    paro_status st = rot_create_128(out, in, K, 2 * P, K ? p128.data() : nullptr, K ? t128.data() : nullptr, alpha);
+    if (st == PARO_OK) (*out)->dev.group = 64;
+    return st;
+}
+
 paro_status paro_rot_destroy(paro_rot* r) {
     g_err[0] = 0;
     if (!r) return PARO_OK;
@@ -331,33 +376,39 @@ paro_status paro_rotate(const paro_rot* r, const void* X, void* Xr, int64_t T, p
     return e == cudaSuccess ? PARO_OK : cuda_fail(e, "rotate launch");
 }
 
-paro_status paro_pack_size(int64_t in, int64_t out, size_t* qb, size_t* sb, size_t* zb) {
+paro_status paro_pack_size_ex(int64_t in, int64_t out, int group, size_t* qb, size_t* sb, size_t* zb) {
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
+    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
     if (!qb || !sb || !zb) return fail(PARO_ERR_ARG, "null size pointer");
+    const int64_t G = in / group;
     *qb = (size_t)(in * out / 2);
-    *sb = (size_t)((out / 16) * (in / 128) * 8 * 4);
-    const int64_t G = in / 128;
+    *sb = (size_t)((out / 16) * G * 8 * 4);
     *zb = (size_t)((out / 16) * (G + (G & 1)) * 8);
     return PARO_OK;
 }
 
-paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t* z, int64_t in, int64_t out,
-                              void* qw, void* sp, void* zp, paro_stream stream) {
+paro_status paro_pack_size(int64_t in, int64_t out, size_t* qb, size_t* sb, size_t* zb) {
+    return paro_pack_size_ex(in, out, 128, qb, sb, zb);
+}
+
+paro_status paro_pack_weights_ex(const uint8_t* q, const uint16_t* s, const uint8_t* z, int64_t in, int64_t out,
+                                 int group, void* qw, void* sp, void* zp, paro_stream stream) {
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
+    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
     if (!q || !s || !z || !qw || !sp || !zp) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(qw) || !aligned16(sp) || !aligned16(zp)) return fail(PARO_ERR_ARG, "outputs must be 16-byte aligned");
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (!is_unregistered_host(q) && !is_unregistered_host(s) && !is_unregistered_host(z)) {
-        cudaError_t e = paro::launch_pack(q, s, z, in, out, qw, sp, zp, cs);
+        cudaError_t e = paro::launch_pack(q, s, z, in, out, group, qw, sp, zp, cs);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "pack launch");
     }
     // host inputs: stage the logical tensors in one temporary device buffer
     // (offline step; synchronous on `stream`)
-    const size_t G = (size_t)(in / 128);
+    const size_t G = (size_t)(in / group);
     const size_t nq = (size_t)in * (size_t)out, ns = (size_t)out * G * 2, nz = (size_t)out * G;
     const size_t oq = 0, os_ = round256(nq), oz = os_ + round256(ns), total = oz + round256(nz);
     char* tmp = nullptr;
@@ -368,22 +419,33 @@ paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t
     if (e == cudaSuccess) e = cudaMemcpyAsync(tmp + oz, z, nz, cudaMemcpyDefault, cs);
     if (e == cudaSuccess)
         e = paro::launch_pack(reinterpret_cast<const uint8_t*>(tmp + oq), reinterpret_cast<const uint16_t*>(tmp + os_),
-                              reinterpret_cast<const uint8_t*>(tmp + oz), in, out, qw, sp, zp, cs);
+                              reinterpret_cast<const uint8_t*>(tmp + oz), in, out, group, qw, sp, zp, cs);
     const cudaError_t e2 = cudaStreamSynchronize(cs);
     cudaFree(tmp);
     if (e != cudaSuccess) return cuda_fail(e, "pack from host memory");
     return e2 == cudaSuccess ? PARO_OK : cuda_fail(e2, "pack from host memory (synchronize)");
 }
 
-paro_status paro_dequant(const void* qw, const void* sp, const void* zp, int64_t in, int64_t out, void* W,
-                         paro_stream stream) {
+paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t* z, int64_t in, int64_t out,
+                              void* qw, void* sp, void* zp, paro_stream stream) {
+    return paro_pack_weights_ex(q, s, z, in, out, 128, qw, sp, zp, stream);
+}
+
+paro_status paro_dequant_ex(const void* qw, const void* sp, const void* zp, int64_t in, int64_t out, int group,
+                            void* W, paro_stream stream) {
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
+    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
     if (!qw || !sp || !zp || !W) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(qw) || !aligned16(sp) || !aligned16(W)) return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
-    cudaError_t e = paro::launch_dequant(qw, sp, zp, in, out, W, static_cast<cudaStream_t>(stream));
+    cudaError_t e = paro::launch_dequant(qw, sp, zp, in, out, group, W, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PARO_OK : cuda_fail(e, "dequant launch");
+}
+
+paro_status paro_dequant(const void* qw, const void* sp, const void* zp, int64_t in, int64_t out, void* W,
+                         paro_stream stream) {
+    return paro_dequant_ex(qw, sp, zp, in, out, 128, W, stream);
 }
 
 paro_status paro_quantize_weights(const paro_rot* r, const void* W, int64_t out, uint8_t* q, uint16_t* s,
@@ -407,12 +469,20 @@ paro_status paro_linear_workspace_size(int64_t T, int64_t in, int64_t out, size_
     return PARO_OK;
 }
 
-paro_status paro_linear_bias(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
-                             const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws,
-                             size_t ws_bytes, paro_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// The layer: fp16 Y, or (y_fp32) the unrounded fp32 sums of a row-parallel slice.
+paro_status linear_impl(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
+                        const void* bias, int group, void* Y, int64_t T, int64_t in, int64_t out, void* ws,
+                        size_t ws_bytes, paro_stream stream, bool y_fp32) {
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
+    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
+    if (r && r->dev.group != group)
+        return fail(PARO_ERR_ARG, "rotation prepared for group %d, weights quantised with group %d", r->dev.group, group);
     if (T < 0) return fail(PARO_ERR_ARG, "tokens=%lld < 0", (long long)T);
     if (T == 0) return PARO_OK;
     if (r && r->dev.in != in) return fail(PARO_ERR_ARG, "rotation prepared for in=%lld, layer has in=%lld", (long long)r->dev.in, (long long)in);
@@ -428,7 +498,7 @@ paro_status paro_linear_bias(const paro_rot* r, const void* X, const void* qw, c
     const paro::RotDev* rd = r ? &r->dev : nullptr;
     cudaError_t e;
     if (T <= 16) {   // decode rotation kernel into ws, then the int4 decode kernel
-        e = paro::launch_gemv(rd, X, qw, sp, zp, bias, Y, T, in, out, ws, s);
+        e = paro::launch_gemv(rd, X, qw, sp, zp, bias, Y, T, in, out, group, ws, s, y_fp32);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
     // X' = X T^-1 into the workspace, then the tensor-core GEMM as a
@@ -439,8 +509,41 @@ paro_status paro_linear_bias(const paro_rot* r, const void* X, const void* qw, c
         if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
         src = ws;
     }
-    e = paro::launch_gemm(src, qw, sp, zp, bias, Y, T, in, out, s);
+    e = paro::launch_gemm(src, qw, sp, zp, bias, Y, T, in, out, group, s, y_fp32);
     return e == cudaSuccess ? PARO_OK : cuda_fail(e, "prefill launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+paro_status paro_linear_ex(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
+                           const void* bias, int group, void* Y, int64_t T, int64_t in, int64_t out, void* ws,
+                           size_t ws_bytes, paro_stream stream) {
+    return linear_impl(r, X, qw, sp, zp, bias, group, Y, T, in, out, ws, ws_bytes, stream, false);
+}
+
+paro_status paro_linear_partial(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
+                                int group, float* Yf, int64_t T, int64_t in, int64_t out, void* ws, size_t ws_bytes,
+                                paro_stream stream) {
+    return linear_impl(r, X, qw, sp, zp, nullptr, group, Yf, T, in, out, ws, ws_bytes, stream, true);
+}
+
+paro_status paro_finalize(const float* Yf, const void* bias, void* Y, int64_t T, int64_t out, paro_stream stream) {
+    g_err[0] = 0;
+    if (T < 0 || out <= 0 || out % 16) return fail(PARO_ERR_ARG, "tokens=%lld, out_features=%lld", (long long)T, (long long)out);
+    if (T == 0) return PARO_OK;
+    if (!Yf || !Y) return fail(PARO_ERR_ARG, "null pointer");
+    if (!aligned16(Yf) || !aligned16(Y)) return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return fail(PARO_ERR_ARG, "bias must be 2-byte aligned");
+    cudaError_t e = paro::launch_finalize(Yf, bias, Y, T, out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARO_OK : cuda_fail(e, "finalize launch");
+}
+
+paro_status paro_linear_bias(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp,
+                             const void* bias, void* Y, int64_t T, int64_t in, int64_t out, void* ws,
+                             size_t ws_bytes, paro_stream stream) {
+    return paro_linear_ex(r, X, qw, sp, zp, bias, 128, Y, T, in, out, ws, ws_bytes, stream);
 }
 
 paro_status paro_linear(const paro_rot* r, const void* X, const void* qw, const void* sp, const void* zp, void* Y,

@@ -20,8 +20,8 @@ def _record(what, value, bound):
     conftest.PARITY.append((test, what, float(value), bound))
 
 
-def check_rotation(got16, x, pairs, theta, alpha):
-    ref = O.rotate_activations(x, pairs, theta, alpha)
+def check_rotation(got16, x, pairs, theta, alpha, group=128):
+    ref = O.rotate_activations(x, pairs, theta, alpha, group)
     fl, lit = O.rotation_rel_error(got16.astype(np.float64), ref)
     _record("X' rel err (floored 1% group max)", fl, ROT_TOL)
     _record("X' rel err (literal, ref != 0)", lit, "reported")
@@ -36,14 +36,14 @@ def output_bound(y, ref, x16):
     return np.maximum(ABS_TOL, np.abs(x16 - ref) + half + ACC_BUDGET)
 
 
-def check_linear(y16, x, pairs, theta, alpha, q, s, z, bias=None):
+def check_linear(y16, x, pairs, theta, alpha, q, s, z, bias=None, group=128):
     if pairs is None:                       # unrotated layer: theta = 0, alpha = 1
-        pairs, theta, alpha = synth.rotation_params(x.shape[1], 1, 0)
+        pairs, theta, alpha = synth.rotation_params(x.shape[1], 1, 0, group=group)
         theta = np.zeros_like(theta)
         alpha = np.ones_like(alpha)
-    ref = O.linear(x, pairs, theta, alpha, q, s, z, bias=bias)
-    x16 = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, round_output=False, bias=bias)
-    floor = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, round_output=True, bias=bias)
+    ref = O.linear(x, pairs, theta, alpha, q, s, z, group=group, bias=bias)
+    x16 = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, group=group, round_output=False, bias=bias)
+    floor = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, group=group, round_output=True, bias=bias)
     y = y16.astype(np.float64)
     rel, mx = O.output_errors(y, ref)
     bound = output_bound(y, ref, x16)

@@ -72,4 +72,16 @@ def test_wait_selftest_limit_checked_before_launch(L):
 
 def test_unsupported_group(L):
     h = ctypes.c_void_p()
-    assert L.paro_rot_create(ctypes.byref(h), 256, 64, 8, 32, None, None, None) == 2
+    assert L.paro_rot_create(ctypes.byref(h), 512, 256, 8, 32, None, None, None) == 2
+    assert L.paro_rot_create(ctypes.byref(h), 256, 64, 8, 33, None, None, None) == 1      # P > group / 2
+    b = ctypes.c_size_t()
+    assert L.paro_pack_size_ex(4096, 64, 256, ctypes.byref(b), ctypes.byref(b), ctypes.byref(b)) == 2
+
+
+def test_pack_size_group_64(L):
+    from rotated_w4_linear_b200 import binding
+    qb, sb, zb = binding.paro_pack_size(4096, 6144, 64)
+    assert qb == 4096 * 6144 // 2
+    assert sb == 6144 // 16 * 64 * 8 * 4 and zb == 6144 // 16 * 64 * 8
+    # 0.5 + 2/64 + 0.5/64 bytes per weight
+    assert (qb + sb + zb) / (4096 * 6144) == pytest.approx(0.5 + 2 / 64 + 0.5 / 64)

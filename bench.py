@@ -42,15 +42,24 @@ MODELS = {
 }
 PROJ = MODELS["llama3-8b"]
 K_LAYERS = 8
-GROUP = 128
+GROUP = 128          # channels per quantisation (and rotation) group; --group changes it
 
 
-def weight_bytes(n_in, n_out):
-    return n_in * n_out // 2 + (n_out * n_in // GROUP) * 2 + (n_out * n_in // GROUP) // 2
+def weight_bytes(n_in, n_out, group=None):
+    g = group or GROUP
+    return n_in * n_out // 2 + (n_out * n_in // g) * 2 + (n_out * n_in // g) // 2
 
 
-def rot_param_bytes(n_in, K=K_LAYERS, P=64):
+def rot_param_bytes(n_in, K=K_LAYERS, P=None):
+    P = P or GROUP // 2
     return K * (n_in // GROUP) * P * (8 + 2) + 4 * n_in
+
+
+def linear(B, rot, x, qw, sp, zp, n_out, Y=None, ws=None):
+    """The layer call: paro_linear for group 128, paro_linear_ex otherwise."""
+    if GROUP == 128:
+        return B.paro_linear(rot, x, qw, sp, zp, n_out, Y=Y, ws=ws)
+    return B.paro_linear_ex(rot, x, qw, sp, zp, n_out, group=GROUP, Y=Y, ws=ws)
 
 
 def call_bytes(T, n_in, n_out):
@@ -208,21 +217,22 @@ def cpu_baseline(tokens: int, budget_s: float = 12.0, torch=None, B=None):
     par = {"max_abs_dY": 0.0, "format_floor": 0.0, "rel_fro": 0.0, "max_abs_Y": 0.0}
     for i, (name, n_in, n_out) in enumerate(PROJ * 16):
         seed = synth.layer_seed(2, i % len(PROJ))
-        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
-        q, s, z = synth.w4_codes(n_out, n_in, seed)
+        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed, pairs_per_group=GROUP // 2, group=GROUP)
+        q, s, z = synth.w4_codes(n_out, n_in, seed, group=GROUP)
         x = synth.activations(tokens, n_in, seed)
         t0 = time.perf_counter()
-        y_ref = O.linear(x, pairs, theta, alpha, q, s, z)
+        y_ref = O.linear(x, pairs, theta, alpha, q, s, z, group=GROUP)
         t_total += time.perf_counter() - t0
         done_bytes += call_bytes(tokens, n_in, n_out)
         n_calls += 1
         names.append(name)
         if B is not None and i < len(PROJ):
-            rot = B.paro_rot_create(pairs, theta, alpha)
-            qw, sp, zp = B.paro_pack_weights(torch.from_numpy(q), torch.from_numpy(s), torch.from_numpy(z))
-            y = B.paro_linear(rot, torch.from_numpy(x).cuda(), qw, sp, zp, n_out).cpu().numpy().astype(np.float64)
+            rot = B.paro_rot_create(pairs, theta, alpha, group=GROUP)
+            qw, sp, zp = B.paro_pack_weights(torch.from_numpy(q), torch.from_numpy(s), torch.from_numpy(z),
+                                             group=GROUP)
+            y = linear(B, rot, torch.from_numpy(x).cuda(), qw, sp, zp, n_out).cpu().numpy().astype(np.float64)
             rot.close()
-            floor = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z).astype(np.float64)
+            floor = O.linear_fp16_pipeline(x, pairs, theta, alpha, q, s, z, group=GROUP).astype(np.float64)
             rel, mx = O.output_errors(y, y_ref)
             par["max_abs_dY"] = max(par["max_abs_dY"], mx)
             par["rel_fro"] = max(par["rel_fro"], rel)
@@ -256,15 +266,15 @@ def run_reference(args, rank: int, world: int):
     inputs = []
     for i, (name, n_in, n_out) in enumerate(PROJ):
         seed = synth.layer_seed(2, i)
-        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
-        q, s_, z = synth.w4_codes(n_out // 16, n_in, seed)
+        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed, pairs_per_group=GROUP // 2, group=GROUP)
+        q, s_, z = synth.w4_codes(n_out // 16, n_in, seed, group=GROUP)
         x = synth.activations(args.tokens, n_in, seed)
         inputs.append((x, pairs, theta, alpha, q, s_, z))
     times = []
     for k in range(args.warmup + args.steps):
         t0 = time.perf_counter()
         for inp in inputs:
-            O.linear(*inp)
+            O.linear(*inp, group=GROUP)
         if k >= args.warmup:
             times.append(time.perf_counter() - t0)
     sample_bytes = sum(call_bytes(args.tokens, i, o // 16) for _, i, o in PROJ)
@@ -283,8 +293,8 @@ def run_reference(args, rank: int, world: int):
 
 def config(args):
     shapes = ", ".join(f"{n} {i}x{o}" for n, i, o in PROJ)
-    return {"workload": f"{getattr(args, 'model', 'llama3-8b')} decoder-layer W4G128 linears ({shapes}), "
-                        f"decode {args.tokens} tokens, K={K_LAYERS} rotation layers x 64 pairs/group",
+    return {"workload": f"{getattr(args, 'model', 'llama3-8b')} decoder-layer W4G{GROUP} linears ({shapes}), "
+                        f"decode {args.tokens} tokens, K={K_LAYERS} rotation layers x {GROUP // 2} pairs/group",
             "tokens": args.tokens, "layers_per_step": args.layers, "rotation_layers": K_LAYERS,
             "group": GROUP, "l2": f"inputs larger than L2: {args.layers} distinct layers per step",
             "parallelism": f"replicas x{args.gpus}"}
@@ -334,7 +344,7 @@ def rotate_result(torch, B, local, T, K, P, steps, warmup, n_in=4096):
                          "frac": nbytes / per / 1e9 / hbm_peak, "traffic": None, "kernel": kern,
                          "bytes_per_call": nbytes, "peak_source": f"{kind} hbm_gbs"},
             "copies": copies, "l2": "inputs larger than L2 (distinct copies per pass)" if 4 * T * n_in * copies > 126e6
-            else "inputs smaller than L2", "clocks": clk.summary()}
+            else "inputs smaller than L2", "clocks": clk.summary(), "fault_code": B.paro_fault_status(clear=True)}
 
 
 def bench_rotate(args, torch, B, local):
@@ -356,10 +366,10 @@ def prefill_result(torch, B, local, T, steps, warmup, model):
     calls = []
     for i, (name, n_in, n_out) in enumerate(MODELS[model]):
         seed = synth.layer_seed(3, i)
-        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
-        rot = B.paro_rot_create(pairs, theta, alpha)
+        pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed, pairs_per_group=GROUP // 2, group=GROUP)
+        rot = B.paro_rot_create(pairs, theta, alpha, group=GROUP)
         w = torch.from_numpy(synth.weight(n_out, n_in, seed)).to(dev)
-        qw, sp, zp = B.paro_pack_weights(*B.paro_quantize_weights(rot, w))
+        qw, sp, zp = B.paro_pack_weights(*B.paro_quantize_weights(rot, w), group=GROUP)
         del w
         x = torch.from_numpy(synth.activations(T, n_in, seed)).to(dev)
         calls.append(dict(rot=rot, n_in=n_in, n_out=n_out, qw=qw, sp=sp, zp=zp, x=x,
@@ -368,8 +378,8 @@ def prefill_result(torch, B, local, T, steps, warmup, model):
 
     def step(rotate=True):
         for p in calls:
-            B.paro_linear(p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
-                          Y=p["y"], ws=p["ws"])
+            linear(B, p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"], Y=p["y"],
+                   ws=p["ws"])
 
     def rotations():
         for p in calls:
@@ -420,7 +430,8 @@ def prefill_result(torch, B, local, T, steps, warmup, model):
                         "peak_source": f"{kind} bf16_tflops_sustained (fp16 and bf16 share the dense tensor rate)"},
            "note": "the unrotated control reads X from HBM; the rotated layer's GEMM reads X' that the rotation "
                    "just wrote, partly from L2, so the overhead can come out below zero",
-           "l2": "inputs larger than L2", "clocks": clk.summary()}
+           "l2": "inputs larger than L2", "clocks": clk.summary(),
+           "fault_code": B.paro_fault_status(clear=True)}
     del graphs
     for p in calls:
         p["rot"].close()
@@ -449,12 +460,15 @@ def main():
                          "prefill: one layer's projections at --tokens (tensor-core GEMM)")
     ap.add_argument("--model", default="llama3-8b", choices=sorted(MODELS),
                     help="decoder-layer shapes (the headline line is llama3-8b)")
+    ap.add_argument("--group", type=int, default=128, choices=[64, 128, 256],
+                    help="channels per quantisation and rotation group (the headline is 128)")
     ap.add_argument("--rot-k", type=int, default=8)
     ap.add_argument("--rot-pairs", type=int, default=64)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    global PROJ
+    global PROJ, GROUP
     PROJ = MODELS[args.model]
+    GROUP = args.group
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -484,11 +498,12 @@ def main():
         projs = []
         for i, (name, n_in, n_out) in enumerate(PROJ):
             seed = synth.layer_seed(2, 100 * (rank * args.layers + l) + i)
-            pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed)
-            rot = B.paro_rot_create(pairs, theta, alpha)
+            pairs, theta, alpha = synth.rotation_params(n_in, K_LAYERS, seed, pairs_per_group=GROUP // 2,
+                                                        group=GROUP)
+            rot = B.paro_rot_create(pairs, theta, alpha, group=GROUP)
             w = torch.from_numpy(synth.weight(n_out, n_in, seed)).to(dev)
             q, s, z = B.paro_quantize_weights(rot, w)
-            qw, sp, zp = B.paro_pack_weights(q, s, z)
+            qw, sp, zp = B.paro_pack_weights(q, s, z, group=GROUP)
             del w, q, s, z
             x = torch.from_numpy(synth.activations(T, n_in, seed)).to(dev)
             y = torch.empty((T, n_out), dtype=torch.float16, device=dev)
@@ -502,8 +517,8 @@ def main():
 
     def step(rotate=True):
         for p in calls:
-            B.paro_linear(p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
-                          Y=p["y"], ws=p["ws"])
+            linear(B, p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"], Y=p["y"],
+                   ws=p["ws"])
 
     # The step is captured once into a CUDA graph (a decode engine replays its
     # step the same way); replays remove the host's per-call launch cost from
@@ -558,8 +573,8 @@ def main():
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 for p in sel:
-                    B.paro_linear(p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
-                                  Y=p["y"], ws=p["ws"])
+                    linear(B, p["rot"] if rotate else None, p["x"], p["qw"], p["sp"], p["zp"], p["n_out"],
+                           Y=p["y"], ws=p["ws"])
             g.replay()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -613,7 +628,7 @@ def main():
         if st["used"]:
             stream.wait_event(st["ev_out"])         # the set's previous outputs are on the host
         for p, x_, y_ in zip(calls, st["xs"], st["ys"]):
-            B.paro_linear(p["rot"], x_, p["qw"], p["sp"], p["zp"], p["n_out"], Y=y_, ws=p["ws"])
+            linear(B, p["rot"], x_, p["qw"], p["sp"], p["zp"], p["n_out"], Y=y_, ws=p["ws"])
         st["ev_done"].record(stream)
         with torch.cuda.stream(d2h_stream):        # outputs: one copy
             d2h_stream.wait_event(st["ev_done"])
@@ -638,6 +653,8 @@ def main():
     elapsed, e2e_elapsed, kern_s = max_over_ranks(dist, [elapsed, e2e_elapsed, kern_s], dev)
     line = decode_line(args, world, elapsed, e2e_elapsed, kern_s, step_bytes, gemv_bytes, len(calls),
                        hbm_peak, peak_kind, h2d, d2h, per_proj, n_launch, clocks)
+    # a bounded wait that ran out would void the numbers: the fault word must read 0
+    line["fault_code"] = B.paro_fault_status(clear=True)
     del g_step, g_gemv
     for projs in layers:
         for p in projs:

@@ -57,9 +57,10 @@ typedef struct paro_rot paro_rot;
 
 /* Validate and prepare the scaled pairwise rotation T of one layer and upload
  * it to the current device (setup; allocates device memory; synchronous).
- *   in_features      multiple of 128
- *   group            channels per quantisation group: 128 or 64 (256 is not
- *                    supported: PARO_ERR_UNSUPPORTED)
+ *   in_features      multiple of 128 (of 256 for group 256)
+ *   group            channels per quantisation group: 128, 64 or 256 (others:
+ *                    PARO_ERR_UNSUPPORTED). With 256 every batch size rotates
+ *                    on the tensor cores (no Givens tables are built).
  *   K                number of rotation layers, 0..16 (K = 0: T = diag(alpha))
  *   pairs_per_group  P, 1..group/2 active pairs per (layer, group)
  *   pairs_host       int16 [K][in/group][P][2], group-local channel indices
@@ -90,10 +91,12 @@ paro_status paro_rotate(const paro_rot* rot, const void* X_dev, void* Xr_dev,
 paro_status paro_pack_size(int64_t in_features, int64_t out_features,
                            size_t* qweight_bytes, size_t* scales_bytes, size_t* zeros_bytes);
 
-/* The same for a quantisation group of `group` channels (128 or 64; the
- * format above is group 128): one scale word and one zero byte per group of
- * each 16-row block's row pairs. Paper: the group size as a speed/accuracy
- * knob (CSDN article, section 5.2). */
+/* The same for a quantisation group of `group` channels (128, 64 or 256;
+ * the format above is group 128): one scale word and one zero byte per group
+ * of each 16-row block's row pairs. Group 256 is stored in the group-128
+ * format, each group's scale and zero repeated for its two 128-channel
+ * halves. Paper: the group size as a speed/accuracy knob (CSDN article,
+ * section 5.2). */
 paro_status paro_pack_size_ex(int64_t in_features, int64_t out_features, int group,
                               size_t* qweight_bytes, size_t* scales_bytes, size_t* zeros_bytes);
 
@@ -116,8 +119,8 @@ paro_status paro_pack_weights(const uint8_t* q, const uint16_t* s, const uint8_t
                               void* qweight_dev, void* scales_dev, void* zeros_dev,
                               paro_stream stream);
 
-/* paro_pack_weights for a quantisation group of `group` channels (128 or 64):
- * s and z are [out][in/group]; sizes from paro_pack_size_ex. */
+/* paro_pack_weights for a quantisation group of `group` channels (128, 64 or
+ * 256): s and z are [out][in/group]; sizes from paro_pack_size_ex. */
 paro_status paro_pack_weights_ex(const uint8_t* q, const uint16_t* s, const uint8_t* z,
                                  int64_t in_features, int64_t out_features, int group,
                                  void* qweight_dev, void* scales_dev, void* zeros_dev,
@@ -130,13 +133,13 @@ paro_status paro_dequant(const void* qweight_dev, const void* scales_dev, const 
                          int64_t in_features, int64_t out_features, void* W_dev,
                          paro_stream stream);
 
-/* paro_dequant for the format of paro_pack_weights_ex with `group` (128 or 64). */
+/* paro_dequant for the format of paro_pack_weights_ex with `group` (128, 64 or 256). */
 paro_status paro_dequant_ex(const void* qweight_dev, const void* scales_dev, const void* zeros_dev,
                             int64_t in_features, int64_t out_features, int group, void* W_dev,
                             paro_stream stream);
 
 /* Offline converter: W' = T W along the input axis (fp64), then asymmetric
- * RTN per input group of the handle's group size (128 or 64):
+ * RTN per input group of the handle's group size (128, 64 or 256):
  * s = fp16((max-min)/15) floored at 2^-14,
  * z = clamp(rint(-min/s), 0, 15), q = clamp(rint(w/s) + z, 0, 15).
  *   W_dev  fp16 [out][in] (PyTorch orientation); outputs q_dev uint8 [out][in],
@@ -187,7 +190,7 @@ paro_status paro_linear_bias(const paro_rot* rot, const void* X_dev,
                              paro_stream stream);
 
 /* The general form of the layer: paro_linear_bias with weights quantised in
- * groups of `group` channels (128 or 64, packed by paro_pack_weights_ex).
+ * groups of `group` channels (128, 64 or 256, packed by paro_pack_weights_ex).
  * A rotation handle, if given, must have been prepared with the same group
  * (else PARO_ERR_ARG). paro_linear and paro_linear_bias are this call with
  * group 128. Paper: CSDN article, section 2.1 (Y = (X T^-1)(T W) + b) and
@@ -259,10 +262,12 @@ paro_status paro_linear_once(const void* X_dev, const int16_t* pairs_host, const
                              const void* zeros_dev, void* Y_dev, int64_t tokens, int64_t in_features,
                              int64_t out_features, int K, int pairs_per_group, paro_stream stream);
 
-/* Fault word of the current device: 0, or the code of a bounded wait inside
- * a tensor-core kernel that ran out (about 2 s) because a pipeline stage
- * never arrived: 1 TMA producer, 2 MMA issuer, 3 dequantisation, 4 epilogue,
- * 5 a drain before exit, 6 the self-test below. The CTA that saw it raises an
+/* Fault word of the current device: 0, or the code of the first bounded wait
+ * inside a tensor-core kernel that ran out (about 2 s) because a pipeline
+ * stage never arrived: the kernel (0 prefill GEMM, 10 tensor-core rotation,
+ * 20 its 256-channel form) plus the role (1 TMA producer, 2 MMA issuer,
+ * 3 dequantisation, 4 epilogue, 5 a drain before exit); 6 is the self-test
+ * below. The CTA that saw it raises an
  * abort flag in its shared memory: every role stops issuing copies and
  * MMAs, the copies and MMAs already issued are waited for (bounded), tensor
  * memory is released and the CTA exits without storing its tile. The output

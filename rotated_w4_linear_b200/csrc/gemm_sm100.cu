@@ -82,6 +82,12 @@ template <int BN, int STAGES, int DQG, int NACC>
 __global__ void __launch_bounds__(64 + 128 * DQG, 1)
 gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z, const GemmArgs a) {
+    // A dequantisation group waits on its stages' mbarriers by phase parity,
+    // which cannot tell phase u from u + 2: each stage must belong to one
+    // group, so that a group's successive waits on it are one phase apart
+    // (with 2 groups and 5 stages a group could come back to a stage while
+    // the other group's use of it was still in flight, and pass on stale data).
+    static_assert(STAGES % DQG == 0, "every stage must belong to one dequantisation group");
     constexpr uint32_t kBStage = BN * 128;              // BN rows x 64 fp16
     constexpr uint32_t kIdesc = umma_idesc_f16(128, BN);
     constexpr uint32_t kTmemCols = tmem_cols<BN, STAGES, NACC>();

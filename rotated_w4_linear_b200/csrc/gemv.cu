@@ -594,10 +594,16 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     cudaGetDevice(&dev);
     const int K = rot ? rot->K : 0;
     const void* xr = X;
-    if (rot) {
+    bool lane_major = false;
+    if (rot && rot->group == 256) {   // no Givens tables: the tensor-core rotation, natural channel order
+        cudaError_t e = launch_rotate_tc(*rot, X, ws, T, s);
+        if (e != cudaSuccess) return e;
+        xr = ws;
+    } else if (rot) {
         cudaError_t e = launch_rotate_decode(*rot, X, ws, T, s, true);
         if (e != cudaSuccess) return e;
         xr = ws;
+        lane_major = true;
     }
     const GemvPlan p = (T > 8) ? (g64 ? cached_plan<2, 2>(dev, in, out, (int)T, K) : cached_plan<2, 1>(dev, in, out, (int)T, K))
                                : (g64 ? cached_plan<1, 2>(dev, in, out, (int)T, K) : cached_plan<1, 1>(dev, in, out, (int)T, K));
@@ -619,7 +625,7 @@ cudaError_t launch_gemv(const RotDev* rot, const void* X, const void* qw, const 
     a.bias = static_cast<const __half*>(bias);
     a.Y = y_fp32 ? nullptr : static_cast<__half*>(Y);
     a.Yf = y_fp32 ? static_cast<float*>(Y) : nullptr;
-    a.xlm = rot ? 1 : 0;
+    a.xlm = lane_major ? 1 : 0;
     cudaError_t e = (T > 8) ? (g64 ? launch_gemv_t<2, 2>(a, p, dev, s) : launch_gemv_t<2, 1>(a, p, dev, s))
                             : (g64 ? launch_gemv_t<1, 2>(a, p, dev, s) : launch_gemv_t<1, 1>(a, p, dev, s));
     if (e != cudaSuccess) return e;

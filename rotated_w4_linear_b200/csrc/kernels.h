@@ -12,7 +12,9 @@ struct RotDev {
     int G = 0;              // groups of 128 (tables are built per 128 channels)
     int K = 0;              // rotation layers
     int P = 0;              // active pairs per (layer, 128-channel group)
-    int group = 128;        // the layer's group size (64: two groups share each 128-channel table)
+    int group = 128;        // the layer's group size (64: two groups share each 128-channel table;
+                            // 256: G counts 256-channel groups, no Givens tables, mats and rotp64
+                            // hold the 256-channel forms)
     uint8_t* rotq = nullptr;       // [K][G] quad exchange blocks (decode prologue)
     float* inv_alpha = nullptr;    // [in] fp32 1/alpha
     uint8_t* rotp64 = nullptr;     // [K][G] blocks of 128 partner bytes + 128 double2 (converter)
@@ -22,6 +24,9 @@ struct RotDev {
 
 // Bytes of one group's dense rotation image: hi and lo fp16 128 x 128.
 constexpr size_t kRotMatBytes = 4 * 128 * 128;
+// For 256-channel groups, one image per half of the output channels: hi and
+// lo fp16 of 256 (k) x 128 (n).
+constexpr size_t kRotMat256Bytes = 4 * 256 * 128;
 
 // 2-D TMA descriptor of a row-major tensor [outer][inner] (driver entry point).
 bool encode_tma_2d(CUtensorMap* tm, CUtensorMapDataType type, const void* base, uint64_t inner, uint64_t outer,

@@ -34,18 +34,22 @@ __global__ void pack_q_kernel(const uint8_t* __restrict__ q, uint32_t* __restric
     qw[w] = word;
 }
 
+// scales and zeros of G destination groups (of 128 or 64 channels); the
+// logical s, z have Gsrc = G / rep groups per row (rep = 2 for groups of 256,
+// whose scale and zero are repeated for both 128-channel halves)
 __global__ void pack_meta_kernel(const uint16_t* __restrict__ s, const uint8_t* __restrict__ z,
-                                 uint32_t* __restrict__ sp, uint8_t* __restrict__ zp, int G, int64_t n) {
+                                 uint32_t* __restrict__ sp, uint8_t* __restrict__ zp, int G, int rep, int64_t n) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (rb, gi, g)
     if (i >= n) return;
-    const int Gp = G + (G & 1);
+    const int Gp = G + (G & 1), Gsrc = G / rep;
     const int g = (int)(i & 7);
     const int64_t rg = i >> 3;
     const int gi = (int)(rg % G);
     const int64_t rb = rg / G;
     const int64_t r0 = rb * 16 + g, r1 = r0 + 8;
-    sp[i] = (uint32_t)s[r0 * G + gi] | ((uint32_t)s[r1 * G + gi] << 16);
-    const uint8_t zb = (uint8_t)((z[r0 * G + gi] & 0xF) | ((z[r1 * G + gi] & 0xF) << 4));
+    const int gs = gi / rep;
+    sp[i] = (uint32_t)s[r0 * Gsrc + gs] | ((uint32_t)s[r1 * Gsrc + gs] << 16);
+    const uint8_t zb = (uint8_t)((z[r0 * Gsrc + gs] & 0xF) | ((z[r1 * Gsrc + gs] & 0xF) << 4));
     zp[(rb * Gp + gi) * 8 + g] = zb;
     if ((G & 1) && gi == G - 1) zp[(rb * Gp + G) * 8 + g] = 0;   // padding group
 }
@@ -55,11 +59,12 @@ cudaError_t launch_pack(const uint8_t* q, const uint16_t* sc, const uint8_t* z, 
     const int64_t nwords = in * out / 8;
     if (nwords > 0)
         pack_q_kernel<<<(unsigned)((nwords + 255) / 256), 256, 0, s>>>(q, static_cast<uint32_t*>(qw), (int)in, nwords);
-    const int G = (int)(in / group);
+    const int rep = group == 256 ? 2 : 1;                      // group 256: stored as group 128
+    const int G = (int)(in / (group == 256 ? 128 : group));
     const int64_t nm = (out / 16) * G * 8;
     if (nm > 0)
         pack_meta_kernel<<<(unsigned)((nm + 255) / 256), 256, 0, s>>>(sc, z, static_cast<uint32_t*>(scp),
-                                                                      static_cast<uint8_t*>(zp), G, nm);
+                                                                      static_cast<uint8_t*>(zp), G, rep, nm);
     return cudaGetLastError();
 }
 
@@ -184,8 +189,85 @@ __global__ void __launch_bounds__(128) quantize_kernel(const __half* __restrict_
     }
 }
 
+// The same for 256-channel groups: one warp per (output row, group), lane L
+// holding channels 8L..8L+7; fp64 blocks of 256 partner bytes + 256 (a, b).
+__global__ void __launch_bounds__(128) quantize256_kernel(const __half* __restrict__ W, int in, int G, int K,
+                                                          int64_t out, const uint8_t* __restrict__ rotp64,
+                                                          const double* __restrict__ alpha64,
+                                                          uint8_t* __restrict__ q, uint16_t* __restrict__ sc,
+                                                          uint8_t* __restrict__ z) {
+    constexpr int kBlk = 256 + 256 * 16;
+    __shared__ double buf[4][256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t task = (int64_t)blockIdx.x * 4 + warp;
+    if (task >= out * G) return;
+    const int gi = (int)(task % G);
+    const int64_t o = task / G;
+    const int c0 = gi * 256 + 8 * lane;
+    const __half* wr = W + o * in + c0;
+    double v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[r] = __dmul_rn((double)__half2float(wr[r]), alpha64[c0 + r]);
+    double* b = buf[warp];
+    for (int t = 0; t < K; ++t) {
+        const uint8_t* blk = rotp64 + ((size_t)t * G + gi) * kBlk;
+        const uint2 pw = reinterpret_cast<const uint2*>(blk)[lane];
+        const double2* cf = reinterpret_cast<const double2*>(blk + 256) + 8 * lane;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) b[8 * lane + r] = v[r];
+        __syncwarp();
+        double p[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) p[r] = b[((r < 4 ? pw.x : pw.y) >> (8 * (r & 3))) & 0xFF];
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const double2 ab = cf[r];
+            v[r] = __dadd_rn(__dmul_rn(ab.x, v[r]), __dmul_rn(ab.y, p[r]));
+        }
+    }
+    double mn = v[0], mx = v[0];
+#pragma unroll
+    for (int r = 1; r < 8; ++r) {
+        mn = fmin(mn, v[r]);
+        mx = fmax(mx, v[r]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    __half s16 = __double2half(__ddiv_rn(__dsub_rn(mx, mn), 15.0));
+    double sd = (double)__half2float(s16);
+    const double floor_s = 6.103515625e-05;   // 2^-14, smallest normal fp16
+    if (sd < floor_s) {
+        sd = floor_s;
+        s16 = __double2half(floor_s);
+    }
+    const double zd = fmin(fmax(rint(__ddiv_rn(-mn, sd)), 0.0), 15.0);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const uint32_t qd = (uint32_t)fmin(fmax(__dadd_rn(rint(__ddiv_rn(v[r], sd)), zd), 0.0), 15.0);
+        if (r < 4) lo |= qd << (8 * r);
+        else hi |= qd << (8 * (r - 4));
+    }
+    *reinterpret_cast<uint2*>(q + o * in + c0) = make_uint2(lo, hi);
+    if (lane == 0) {
+        sc[o * G + gi] = __half_as_ushort(s16);
+        z[o * G + gi] = (uint8_t)zd;
+    }
+}
+
 cudaError_t launch_quantize(const RotDev& r, const void* W, int64_t out, uint8_t* q, uint16_t* sc, uint8_t* z,
                             cudaStream_t s) {
+    if (r.group == 256) {
+        const int64_t tasks = out * r.G;
+        if (tasks > 0)
+            quantize256_kernel<<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(static_cast<const __half*>(W), (int)r.in,
+                                                                           r.G, r.K, out, r.rotp64, r.alpha64, q, sc, z);
+        return cudaGetLastError();
+    }
     const int64_t tasks = out * r.G;
     if (tasks > 0)
         quantize_kernel<<<(unsigned)((tasks + 3) / 4), 128, 0, s>>>(static_cast<const __half*>(W), (int)r.in, r.G,

@@ -106,6 +106,39 @@ bool is_unregistered_host(const void* p) {
     return a.type == cudaMemoryTypeUnregistered;
 }
 
+// The same for a 256-channel group: M is 256 x 256; per half h of the
+// output channels one 128 KB image of B[n][k] = M[k][128 h + n], n < 128,
+// k < 256: hi then lo, each as four 64-channel quarters of k (128 rows x 128
+// bytes, 128-byte swizzle).
+void dense_group_image_256(const int16_t* pairs, const float* theta, const float* alpha, int K, int P, int G, int g,
+                           uint8_t* out /* [2][128 KB] */) {
+    std::vector<double> M(256 * 256, 0.0);                // M[k * 256 + n]
+    for (int k = 0; k < 256; ++k) M[k * 256 + k] = 1.0 / (double)alpha[g * 256 + k];
+    for (int t = 0; t < K; ++t)
+        for (int p = 0; p < P; ++p) {
+            const size_t base = (((size_t)t * G + g) * P + p);
+            const int i = pairs[2 * base], j = pairs[2 * base + 1];
+            const double c = std::cos((double)theta[base]), sn = std::sin((double)theta[base]);
+            for (int k = 0; k < 256; ++k) {
+                const double vi = M[k * 256 + i], vj = M[k * 256 + j];
+                M[k * 256 + i] = c * vi - sn * vj;
+                M[k * 256 + j] = sn * vi + c * vj;
+            }
+        }
+    for (int h = 0; h < 2; ++h)
+        for (int part = 0; part < 2; ++part)
+            for (int n = 0; n < 128; ++n)
+                for (int k = 0; k < 256; ++k) {
+                    const double m = M[k * 256 + 128 * h + n];
+                    const __half hi = __double2half(m);
+                    const __half v = part == 0 ? hi : __double2half(m - (double)__half2float(hi));
+                    const int q = k >> 6, chunk = (k & 63) >> 3, e = k & 7;
+                    const size_t off = (size_t)h * 131072 + (size_t)part * 65536 + (size_t)q * 16384 +
+                                       (size_t)n * 128 + (size_t)((chunk ^ (n & 7)) << 4) + (size_t)e * 2;
+                    memcpy(out + off, &v, 2);
+                }
+}
+
 }  // namespace
 
 extern "C" {
@@ -314,6 +347,79 @@ paro_status rot_create_128(paro_rot** out, int64_t in, int K, int P, const int16
     return PARO_OK;
 }
 
+// The handle for 256-channel groups: fp64 blocks for the converter (256
+// partner bytes + 256 (a, b) pairs per layer and group) and the dense images
+// for the tensor-core rotation; the Givens kernel's 128-channel tables are
+// not built (every batch size rotates on the tensor cores).
+paro_status rot_create_256(paro_rot** out, int64_t in, int K, int P, const int16_t* pairs, const float* theta,
+                           const float* alpha) {
+    if (in > (1LL << 20)) return fail(PARO_ERR_UNSUPPORTED, "in_features too large");
+    if (!alpha) return fail(PARO_ERR_ARG, "alpha is null");
+    paro_status st = check_device();
+    if (st != PARO_OK) return st;
+    const int G = (int)(in / 256);
+    for (int64_t c = 0; c < in; ++c)
+        if (!std::isfinite(alpha[c]) || alpha[c] == 0.0f)
+            return fail(PARO_ERR_ARG, "alpha[%lld] must be finite and non-zero", (long long)c);
+    constexpr size_t kBlk = 256 + 256 * 16;
+    std::vector<uint8_t> rot64((size_t)K * G * kBlk);
+    for (int t = 0; t < K; ++t)
+        for (int g = 0; g < G; ++g) {
+            uint8_t partner[256];
+            double a64[256], b64[256];
+            bool used[256] = {false};
+            for (int c = 0; c < 256; ++c) { partner[c] = (uint8_t)c; a64[c] = 1.0; b64[c] = 0.0; }
+            for (int p = 0; p < P; ++p) {
+                const size_t base = (((size_t)t * G + g) * P + p);
+                const int i = pairs[2 * base], j = pairs[2 * base + 1];
+                const float th = theta[base];
+                if (i < 0 || i >= 256 || j < 0 || j >= 256)
+                    return fail(PARO_ERR_ARG, "pair (%d,%d) of layer %d group %d leaves the group", i, j, t, g);
+                if (i == j || used[i] || used[j])
+                    return fail(PARO_ERR_ARG, "channel reused within layer %d group %d (pair %d: %d,%d)", t, g, p, i, j);
+                if (!std::isfinite(th)) return fail(PARO_ERR_ARG, "theta of layer %d group %d pair %d is not finite", t, g, p);
+                used[i] = used[j] = true;
+                const double c = std::cos((double)th), sn = std::sin((double)th);
+                partner[i] = (uint8_t)j; a64[i] = c; b64[i] = -sn;
+                partner[j] = (uint8_t)i; a64[j] = c; b64[j] = sn;
+            }
+            uint8_t* b6 = &rot64[((size_t)t * G + g) * kBlk];
+            memcpy(b6, partner, 256);
+            for (int c = 0; c < 256; ++c) {
+                memcpy(b6 + 256 + 16 * c, &a64[c], 8);
+                memcpy(b6 + 256 + 16 * c + 8, &b64[c], 8);
+            }
+        }
+    std::vector<uint8_t> mats((size_t)G * 2 * paro::kRotMat256Bytes);
+    for (int g = 0; g < G; ++g)
+        dense_group_image_256(pairs, theta, alpha, K, P, G, g, &mats[(size_t)g * 2 * paro::kRotMat256Bytes]);
+    std::vector<double> alpha64((size_t)in);
+    for (int64_t c = 0; c < in; ++c) alpha64[c] = (double)alpha[c];
+    const size_t o_rot64 = 0, o_a64 = round256(rot64.size()), o_mats = o_a64 + round256(alpha64.size() * 8);
+    const size_t total = o_mats + round256(mats.size());
+    paro_rot* r = new (std::nothrow) paro_rot();
+    if (!r) return fail(PARO_ERR_ARG, "out of host memory");
+    cudaGetDevice(&r->device);
+    cudaError_t e = cudaMalloc(&r->block, total);
+    if (e != cudaSuccess) { delete r; return cuda_fail(e, "cudaMalloc(rotation tables)"); }
+    char* base = static_cast<char*>(r->block);
+    e = cudaSuccess;
+    if (!rot64.empty()) e = cudaMemcpy(base + o_rot64, rot64.data(), rot64.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + o_a64, alpha64.data(), alpha64.size() * 8, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(base + o_mats, mats.data(), mats.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(r->block); delete r; return cuda_fail(e, "cudaMemcpy(rotation tables)"); }
+    r->dev.in = in;
+    r->dev.G = G;
+    r->dev.K = K;
+    r->dev.P = P;
+    r->dev.group = 256;
+    r->dev.rotp64 = reinterpret_cast<uint8_t*>(base + o_rot64);
+    r->dev.alpha64 = reinterpret_cast<double*>(base + o_a64);
+    r->dev.mats = reinterpret_cast<uint8_t*>(base + o_mats);
+    *out = r;
+    return PARO_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -323,14 +429,16 @@ paro_status paro_rot_create(paro_rot** out, int64_t in, int group, int K, int P,
     g_err[0] = 0;
     if (!out) return fail(PARO_ERR_ARG, "out is null");
     *out = nullptr;
-    if (group != 128 && group != 64)
-        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
-    if (in <= 0 || in % 128)
-        return fail(PARO_ERR_ARG, "in_features=%lld must be a positive multiple of 128", (long long)in);
+    if (group != 128 && group != 64 && group != 256)
+        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 64, 128 and 256 are supported", group);
+    const int unit = group == 256 ? 256 : 128;
+    if (in <= 0 || in % unit)
+        return fail(PARO_ERR_ARG, "in_features=%lld must be a positive multiple of %d", (long long)in, unit);
     if (K < 0 || K > 16) return fail(PARO_ERR_ARG, "K=%d must be in 0..16", K);
     if (K > 0 && (P < 1 || P > group / 2)) return fail(PARO_ERR_ARG, "pairs_per_group=%d must be in 1..%d", P, group / 2);
     if (K > 0 && (!pairs || !theta)) return fail(PARO_ERR_ARG, "pairs/theta is null");
     if (group == 128) return rot_create_128(out, in, K, P, pairs, theta, alpha);
+    if (group == 256) return rot_create_256(out, in, K, P, pairs, theta, alpha);
     // groups of 64: the pairs of 64-channel groups 2h and 2h + 1 (indices
     // 0..63 each) form the 128-channel table h, the second group's indices
     // moved up by 64; a pair cannot leave its 64-channel group
@@ -380,9 +488,11 @@ paro_status paro_pack_size_ex(int64_t in, int64_t out, int group, size_t* qb, si
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
-    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
+    if (group != 128 && group != 64 && group != 256)
+        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 64, 128 and 256 are supported", group);
+    if (group == 256 && in % 256) return fail(PARO_ERR_ARG, "in_features=%lld: group 256 needs a multiple of 256", (long long)in);
     if (!qb || !sb || !zb) return fail(PARO_ERR_ARG, "null size pointer");
-    const int64_t G = in / group;
+    const int64_t G = in / (group == 256 ? 128 : group);     // group 256: stored as group 128
     *qb = (size_t)(in * out / 2);
     *sb = (size_t)((out / 16) * G * 8 * 4);
     *zb = (size_t)((out / 16) * (G + (G & 1)) * 8);
@@ -398,7 +508,9 @@ paro_status paro_pack_weights_ex(const uint8_t* q, const uint16_t* s, const uint
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
-    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
+    if (group != 128 && group != 64 && group != 256)
+        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 64, 128 and 256 are supported", group);
+    if (group == 256 && in % 256) return fail(PARO_ERR_ARG, "in_features=%lld: group 256 needs a multiple of 256", (long long)in);
     if (!q || !s || !z || !qw || !sp || !zp) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(qw) || !aligned16(sp) || !aligned16(zp)) return fail(PARO_ERR_ARG, "outputs must be 16-byte aligned");
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -436,7 +548,9 @@ paro_status paro_dequant_ex(const void* qw, const void* sp, const void* zp, int6
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
-    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
+    if (group != 128 && group != 64 && group != 256)
+        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 64, 128 and 256 are supported", group);
+    if (group == 256) group = 128;                                // stored as group 128
     if (!qw || !sp || !zp || !W) return fail(PARO_ERR_ARG, "null pointer");
     if (!aligned16(qw) || !aligned16(sp) || !aligned16(W)) return fail(PARO_ERR_ARG, "pointers must be 16-byte aligned");
     cudaError_t e = paro::launch_dequant(qw, sp, zp, in, out, group, W, static_cast<cudaStream_t>(stream));
@@ -480,9 +594,13 @@ paro_status linear_impl(const paro_rot* r, const void* X, const void* qw, const 
     g_err[0] = 0;
     paro_status st = check_shape(in, out);
     if (st != PARO_OK) return st;
-    if (group != 128 && group != 64) return fail(PARO_ERR_UNSUPPORTED, "group=%d: 128 and 64 are supported", group);
+    if (group != 128 && group != 64 && group != 256)
+        return fail(PARO_ERR_UNSUPPORTED, "group=%d: 64, 128 and 256 are supported", group);
     if (r && r->dev.group != group)
         return fail(PARO_ERR_ARG, "rotation prepared for group %d, weights quantised with group %d", r->dev.group, group);
+    if (group == 256 && in % 256) return fail(PARO_ERR_ARG, "in_features=%lld: group 256 needs a multiple of 256", (long long)in);
+    // group 256 weights are stored in the group-128 format (each scale and zero repeated)
+    const int fmt_group = group == 256 ? 128 : group;
     if (T < 0) return fail(PARO_ERR_ARG, "tokens=%lld < 0", (long long)T);
     if (T == 0) return PARO_OK;
     if (r && r->dev.in != in) return fail(PARO_ERR_ARG, "rotation prepared for in=%lld, layer has in=%lld", (long long)r->dev.in, (long long)in);
@@ -498,7 +616,7 @@ paro_status linear_impl(const paro_rot* r, const void* X, const void* qw, const 
     const paro::RotDev* rd = r ? &r->dev : nullptr;
     cudaError_t e;
     if (T <= 16) {   // decode rotation kernel into ws, then the int4 decode kernel
-        e = paro::launch_gemv(rd, X, qw, sp, zp, bias, Y, T, in, out, group, ws, s, y_fp32);
+        e = paro::launch_gemv(rd, X, qw, sp, zp, bias, Y, T, in, out, fmt_group, ws, s, y_fp32);
         return e == cudaSuccess ? PARO_OK : cuda_fail(e, "decode launch");
     }
     // X' = X T^-1 into the workspace, then the tensor-core GEMM as a
@@ -509,7 +627,7 @@ paro_status linear_impl(const paro_rot* r, const void* X, const void* qw, const 
         if (e != cudaSuccess) return cuda_fail(e, "rotate launch");
         src = ws;
     }
-    e = paro::launch_gemm(src, qw, sp, zp, bias, Y, T, in, out, group, s, y_fp32);
+    e = paro::launch_gemm(src, qw, sp, zp, bias, Y, T, in, out, fmt_group, s, y_fp32);
     return e == cudaSuccess ? PARO_OK : cuda_fail(e, "prefill launch");
 }
 

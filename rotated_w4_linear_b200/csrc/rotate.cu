@@ -261,7 +261,7 @@ size_t rotate_decode_smem(int K, int T) { return (size_t)K * kRotQBlockBytes + (
 cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s,
                                  bool lane_major) {
     if (T <= 0) return cudaSuccess;
-    if (T > 16) return cudaErrorInvalidValue;
+    if (T > 16 || r.group == 256 || !r.rotq) return cudaErrorInvalidValue;
     // prefetching the next layer's tables pays with several warps per CTA
     // (measured: 2% of the decode step at 16 tokens) but not with one or two
     const int warps = (int)((T + 3) / 4);
@@ -271,7 +271,8 @@ cudaError_t launch_rotate_decode(const RotDev& r, const void* X, void* Xr, int64
 
 cudaError_t launch_rotate(const RotDev& r, const void* X, void* Xr, int64_t T, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    if (T < kRotateTcMinTokens) return launch_rotate_decode(r, X, Xr, T, s);
+    // 256-channel groups have no Givens tables: every batch on the tensor cores
+    if (T < kRotateTcMinTokens && r.group != 256) return launch_rotate_decode(r, X, Xr, T, s);
     return launch_rotate_tc(r, X, Xr, T, s);
 }
 

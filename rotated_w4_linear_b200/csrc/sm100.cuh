@@ -14,8 +14,12 @@ namespace paro {
 // translation unit that includes this header; the library has one).
 static __device__ unsigned int g_paro_fault = 0;
 
+// (kernel offset + role): prefill GEMM 0, tensor-core rotation 10, its
+// 256-channel form 20; roles 1 TMA producer, 2 MMA issuer, 3 dequantisation,
+// 4 epilogue, 5 a drain before exit; 6 the self-test
 enum : unsigned int { kFaultTmaWait = 1, kFaultMmaWait = 2, kFaultDequantWait = 3, kFaultEpilogueWait = 4,
                       kFaultDrainWait = 5, kFaultSelfTest = 6 };
+enum : unsigned int { kFaultGemm = 0, kFaultRotate = 10, kFaultRotate256 = 20 };
 
 // Time limit of a pipeline wait: far above any stage of a correct kernel.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

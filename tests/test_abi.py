@@ -72,10 +72,16 @@ def test_wait_selftest_limit_checked_before_launch(L):
 
 def test_unsupported_group(L):
     h = ctypes.c_void_p()
-    assert L.paro_rot_create(ctypes.byref(h), 512, 256, 8, 32, None, None, None) == 2
+    assert L.paro_rot_create(ctypes.byref(h), 512, 32, 8, 16, None, None, None) == 2
     assert L.paro_rot_create(ctypes.byref(h), 256, 64, 8, 33, None, None, None) == 1      # P > group / 2
+    assert L.paro_rot_create(ctypes.byref(h), 384, 256, 8, 64, None, None, None) == 1     # in % 256
     b = ctypes.c_size_t()
-    assert L.paro_pack_size_ex(4096, 64, 256, ctypes.byref(b), ctypes.byref(b), ctypes.byref(b)) == 2
+    assert L.paro_pack_size_ex(4096, 64, 512, ctypes.byref(b), ctypes.byref(b), ctypes.byref(b)) == 2
+
+
+def test_pack_size_group_256_is_the_group_128_format(L):
+    from rotated_w4_linear_b200 import binding
+    assert binding.paro_pack_size(4096, 6144, 256) == binding.paro_pack_size(4096, 6144, 128)
 
 
 def test_pack_size_group_64(L):

@@ -371,3 +371,38 @@ def test_bounded_wait_runs_out_and_the_context_survives(B):
     rot = B.paro_rot_create(pairs, theta, alpha)
     check_linear(host(B.paro_linear(rot, dev(x), qw, sp, zp, 48)), x, pairs, theta, alpha, q, s, z)
     assert B.paro_fault_status() == 0
+
+
+def test_prefill_graph_replays_keep_the_fault_word_clear(B):
+    """The prefill path (tensor-core rotation, then the GEMM as a programmatic
+    dependent launch) replayed back to back from a CUDA graph: no bounded
+    wait runs out, and every replay gives the first replay's bits."""
+    T, shapes = 2048, [(4096, 6144), (14336, 1024), (4096, 4096)]
+    calls = []
+    for i, (in_f, out_f) in enumerate(shapes):
+        seed = synth.layer_seed(13, i)
+        pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+        q, s, z = synth.w4_codes(out_f, in_f, seed)
+        qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+        calls.append(dict(rot=B.paro_rot_create(pairs, theta, alpha), x=dev(synth.activations(T, in_f, seed)),
+                          qw=qw, sp=sp, zp=zp, out=out_f, y=torch.empty((T, out_f), dtype=torch.float16, device="cuda"),
+                          ws=B.workspace(T, in_f, out_f)))
+
+    def step():
+        for c in calls:
+            B.paro_linear(c["rot"], c["x"], c["qw"], c["sp"], c["zp"], c["out"], Y=c["y"], ws=c["ws"])
+
+    B.paro_fault_status(clear=True)
+    step()
+    torch.cuda.synchronize()
+    first = [c["y"].clone() for c in calls]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(60):
+        g.replay()
+    torch.cuda.synchronize()
+    assert B.paro_fault_status() == 0
+    for c, y0 in zip(calls, first):
+        assert torch.equal(c["y"], y0)
+    del g

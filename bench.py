@@ -71,8 +71,8 @@ def call_bytes(T, n_in, n_out):
 # one ncu capture at 16 tokens of the decode kernel built from the gemv.cu
 # whose SHA-256 prefix is GEMV_TRAFFIC_SOURCE; reported only while gemv.cu is
 # that file (any change to it nulls the figure until it is captured again).
-GEMV_TRAFFIC_PER_LAUNCH_T16 = (13239040 + 8883968 + 61178880 + 30999040) / 4
-GEMV_TRAFFIC_SOURCE = "e96d84dec74edc6e"
+GEMV_TRAFFIC_PER_LAUNCH_T16 = (13244928 + 8886016 + 61185280 + 31004928) / 4
+GEMV_TRAFFIC_SOURCE = "4c0f8d3a1a030105"
 
 
 def gemv_source_sha() -> str:
@@ -84,7 +84,7 @@ def gemv_source_sha() -> str:
 def gemv_traffic(tokens: int, model: str):
     """The captured DRAM traffic per decode launch, if it belongs to this
     workload and to the current kernel source; else None."""
-    if tokens != 16 or model != "llama3-8b" or gemv_source_sha() != GEMV_TRAFFIC_SOURCE:
+    if tokens != 16 or model != "llama3-8b" or GROUP != 128 or gemv_source_sha() != GEMV_TRAFFIC_SOURCE:
         return None
     return GEMV_TRAFFIC_PER_LAUNCH_T16
 
@@ -307,8 +307,9 @@ def rotate_result(torch, B, local, T, K, P, steps, warmup, n_in=4096):
     Algorithmic bytes: X read + X' written + the rotation parameters
     (per pair an fp32 cos/sin pair and two channel bytes, plus 1/alpha)."""
     torch.cuda.set_device(local)
-    pairs, theta, alpha = synth.rotation_params(n_in, K, synth.layer_seed(1, K), pairs_per_group=P)
-    rot = B.paro_rot_create(pairs, theta, alpha)
+    P = GROUP // 2 if P is None else P
+    pairs, theta, alpha = synth.rotation_params(n_in, K, synth.layer_seed(1, K), pairs_per_group=P, group=GROUP)
+    rot = B.paro_rot_create(pairs, theta, alpha, group=GROUP)
     copies = min(64, max(1, (512 << 20) // (4 * T * n_in)))   # > L2 for T >= 256
     xs = [torch.from_numpy(synth.activations(T, n_in, synth.layer_seed(1, c))).cuda() for c in range(copies)]
     ys = [torch.empty_like(x) for x in xs]
@@ -337,8 +338,11 @@ def rotate_result(torch, B, local, T, K, P, steps, warmup, n_in=4096):
     rot.close()
     nbytes = 4 * T * n_in + K * (n_in // GROUP) * P * 10 + 4 * n_in
     hbm_peak, _, kind = peaks()
-    kern = "rotate_tc_kernel (tensor cores)" if T >= 128 else "rotate_kernel / rotate_quad_kernel (Givens)"
-    return {"workload": f"paro_rotate tokens={T} hidden={n_in} K={K} pairs/group={P}",
+    if GROUP == 256:
+        kern = "rotate_tc256_kernel (tensor cores, 256-channel groups)"
+    else:
+        kern = "rotate_tc_kernel (tensor cores)" if T > 16 else "rotate_quad_kernel (Givens)"
+    return {"workload": f"paro_rotate tokens={T} hidden={n_in} K={K} group={GROUP} pairs/group={P}",
             "us_per_call": per * 1e6, "GB/s": nbytes / per / 1e9,
             "roofline": {"bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": nbytes / per / 1e9 / hbm_peak, "traffic": None, "kernel": kern,
@@ -463,7 +467,7 @@ def main():
     ap.add_argument("--group", type=int, default=128, choices=[64, 128, 256],
                     help="channels per quantisation and rotation group (the headline is 128)")
     ap.add_argument("--rot-k", type=int, default=8)
-    ap.add_argument("--rot-pairs", type=int, default=64)
+    ap.add_argument("--rot-pairs", type=int, default=None)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     global PROJ, GROUP
@@ -667,7 +671,7 @@ def main():
     # them on its own GPU, rank 0 reports its figures
     if not args.no_extra:
         xs = min(args.steps, 20)
-        line["rotate"] = rotate_result(torch, B, local, 8192, K_LAYERS, 64, xs, 3)
+        line["rotate"] = rotate_result(torch, B, local, 8192, K_LAYERS, None, xs, 3)
         line["prefill"] = prefill_result(torch, B, local, 8192, xs, 3, args.model)
         torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -243,12 +243,17 @@ gemm_w4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     for (int j = 0; j < 16; ++j) red[j * kRedStride + rloc] = __uint_as_float(r[j]);
                 } else if (row < a.out) {
                     const float b = a.bias ? __half2float(a.bias[row]) : 0.f;
+                    if (a.Yf) {                               // fp32 partial sums (row-parallel)
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = n0 + c0 + j;
-                        if (t < a.T) {
-                            if (a.Yf) a.Yf[(size_t)t * a.out + row] = __uint_as_float(r[j]) + b;
-                            else a.Y[(size_t)t * a.out + row] = __float2half_rn(__uint_as_float(r[j]) + b);
+                        for (int j = 0; j < 16; ++j) {
+                            const int t = n0 + c0 + j;
+                            if (t < a.T) a.Yf[(size_t)t * a.out + row] = __uint_as_float(r[j]) + b;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int t = n0 + c0 + j;
+                            if (t < a.T) a.Y[(size_t)t * a.out + row] = __float2half_rn(__uint_as_float(r[j]) + b);
                         }
                     }
                 }

@@ -406,3 +406,50 @@ def test_prefill_graph_replays_keep_the_fault_word_clear(B):
     for c, y0 in zip(calls, first):
         assert torch.equal(c["y"], y0)
     del g
+
+
+
+def test_decode_calls_of_several_shapes_share_one_workspace(B):
+    """Decode calls whose grids differ in size, one after another on one
+    workspace (eager, then 40 replays of a CUDA graph of them, each rotation
+    a programmatic dependent of the decode kernel before it): no wait runs
+    out, and every output matches the oracle."""
+    T = 16
+    shapes = [(4096, 6144), (4096, 4096), (4096, 28672), (14336, 4096), (640, 272)]
+    calls = []
+    for i, (in_f, out_f) in enumerate(shapes):
+        seed = synth.layer_seed(15, i)
+        pairs, theta, alpha = synth.rotation_params(in_f, 8, seed)
+        q, s, z = synth.w4_codes(out_f, in_f, seed)
+        qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z))
+        x = synth.activations(T, in_f, seed)
+        calls.append(dict(p=(pairs, theta, alpha, q, s, z), x=x, xd=dev(x), rot=B.paro_rot_create(pairs, theta, alpha),
+                          qw=qw, sp=sp, zp=zp, out=out_f,
+                          y=torch.empty((T, out_f), dtype=torch.float16, device="cuda")))
+    ws = B.workspace(T, max(i for i, _ in shapes), max(o for _, o in shapes))
+
+    def step():
+        for c in calls:
+            B.paro_linear(c["rot"], c["xd"], c["qw"], c["sp"], c["zp"], c["out"], Y=c["y"], ws=ws)
+
+    def check():
+        for c in calls:
+            pairs, theta, alpha, q, s, z = c["p"]
+            rows = np.random.default_rng(c["out"]).choice(c["out"], min(c["out"], 96), replace=False)
+            check_linear(host(c["y"])[:, rows], c["x"], pairs, theta, alpha, q[rows], s[rows], z[rows])
+
+    B.paro_fault_status(clear=True)
+    step()
+    torch.cuda.synchronize()
+    check()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for c in calls:
+        c["y"].zero_()
+    for _ in range(40):
+        g.replay()
+    torch.cuda.synchronize()
+    assert B.paro_fault_status() == 0
+    check()
+    del g

@@ -620,6 +620,11 @@ def main():
                          ev_out=torch.cuda.Event(), used=False))
     h2d_stream = torch.cuda.Stream(device=dev)
     d2h_stream = torch.cuda.Stream(device=dev)
+    # the public per-call API of a decode loop: one prepared layer per
+    # projection (weights and workspace checked once, X and Y per call)
+    for p in calls:
+        p["layer"] = B.ParoLinear(p["rot"], p["qw"], p["sp"], p["zp"], p["n_in"], p["n_out"], group=GROUP)
+        p["layer"]._workspace(T)
 
     def e2e_step(k):
         st = sets[k & 1]
@@ -632,7 +637,7 @@ def main():
         if st["used"]:
             stream.wait_event(st["ev_out"])         # the set's previous outputs are on the host
         for p, x_, y_ in zip(calls, st["xs"], st["ys"]):
-            linear(B, p["rot"], x_, p["qw"], p["sp"], p["zp"], p["n_out"], Y=y_, ws=p["ws"])
+            p["layer"](x_, Y=y_)
         st["ev_done"].record(stream)
         with torch.cuda.stream(d2h_stream):        # outputs: one copy
             d2h_stream.wait_event(st["ev_done"])

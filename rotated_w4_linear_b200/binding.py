@@ -318,6 +318,61 @@ def paro_linear_ex(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_fea
     return Y
 
 
+class ParoLinear:
+    """A prepared layer for repeated calls (a decode loop): the rotation
+    handle, the packed weights, the bias and a workspace are checked once
+    here; a call checks only X and Y and hands raw pointers to the same C
+    entry point as paro_linear_ex. The workspace is owned by the object and
+    grows with the largest batch seen, so calls on one object must not
+    overlap on the GPU (one stream, or events), as for paro_linear's
+    workspace. The object keeps references to the tensors it was given."""
+
+    def __init__(self, rot: Optional[Rotation], qw, sp, zp, in_features: int, out_features: int, group: int = 128,
+                 bias: Optional[torch.Tensor] = None, device=None):
+        if rot is not None and (rot.group != group or rot.in_features != in_features):
+            raise ValueError("the rotation was prepared for another group size or input width")
+        self.rot, self.in_features, self.out_features, self.group = rot, int(in_features), int(out_features), group
+        self._tensors = (qw, sp, zp, bias)                 # kept alive for the pointers below
+        self._h = rot.handle if rot is not None else None
+        self._qw, self._sp, self._zp = _dev(qw, torch.uint8, "qweight"), _dev(sp, torch.uint8, "scales"), \
+            _dev(zp, torch.uint8, "zeros")
+        self._b = None
+        if bias is not None:
+            if bias.numel() != out_features:
+                raise ValueError("bias must have out_features elements")
+            self._b = _dev(bias, torch.float16, "bias")
+        self.device = qw.device if device is None else torch.device(device)
+        self._ws = None
+        self._ws_tokens = 0
+        self._f = lib().paro_linear_ex
+
+    def _workspace(self, T: int) -> None:
+        if T > self._ws_tokens:
+            self._ws = workspace(T, self.in_features, self.out_features, self.device)
+            self._ws_tokens = T
+
+    def __call__(self, X: torch.Tensor, Y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        T = X.shape[0]
+        if not X.is_cuda or X.dtype is not torch.float16 or not X.is_contiguous() or X.dim() != 2 \
+                or X.shape[1] != self.in_features:
+            raise TypeError(f"X must be a contiguous fp16 CUDA tensor [tokens][{self.in_features}]")
+        if Y is None:
+            Y = torch.empty((T, self.out_features), dtype=torch.float16, device=X.device)
+        elif not Y.is_cuda or Y.dtype is not torch.float16 or not Y.is_contiguous() or Y.numel() != T * self.out_features:
+            raise TypeError(f"Y must be a contiguous fp16 CUDA tensor [tokens][{self.out_features}]")
+        if T > self._ws_tokens:
+            self._workspace(T)
+        if stream is None:
+            sp = int(_raw_stream(X.get_device())) if _raw_stream is not None else _stream(None, X.device)
+        else:
+            sp = _stream(stream, X.device)
+        st = self._f(self._h, X.data_ptr(), self._qw, self._sp, self._zp, self._b, self.group, Y.data_ptr(), T,
+                     self.in_features, self.out_features, self._ws.data_ptr(), self._ws.numel(), sp)
+        if st != PARO_OK:
+            _check("paro_linear_ex", st)
+        return Y
+
+
 def paro_linear_partial(rot: Optional[Rotation], X: torch.Tensor, qw, sp, zp, out_features: int, group: int = 128,
                         Yf: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                         stream=None) -> torch.Tensor:

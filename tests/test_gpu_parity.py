@@ -453,3 +453,28 @@ def test_decode_calls_of_several_shapes_share_one_workspace(B):
     assert B.paro_fault_status() == 0
     check()
     del g
+
+
+@pytest.mark.parametrize("group", [128, 64])
+def test_prepared_layer_matches_the_oracle(B, group):
+    """ParoLinear (weights, bias and workspace checked once, the workspace
+    grown with the batch) over decode and prefill batches, against the
+    oracle; a wrongly shaped X is refused before any launch."""
+    in_f, out_f = 640, 272
+    seed = synth.layer_seed(16, group)
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed, pairs_per_group=group // 2, group=group)
+    q, s, z = synth.w4_codes(out_f, in_f, seed, group=group)
+    qw, sp, zp = B.paro_pack_weights(dev(q), dev(s), dev(z), group=group)
+    b = (np.random.default_rng(seed).standard_normal(out_f) * 2).astype(np.float16)
+    rot = B.paro_rot_create(pairs, theta, alpha, group=group)
+    layer = B.ParoLinear(rot, qw, sp, zp, in_f, out_f, group=group, bias=dev(b))
+    for T in (1, 16, 5, 300):
+        x = synth.activations(T, in_f, seed + T)
+        y = torch.empty((T, out_f), dtype=torch.float16, device="cuda")
+        layer(dev(x), Y=y)
+        check_linear(host(y), x, pairs, theta, alpha, q, s, z, bias=b, group=group)
+    with pytest.raises(TypeError):
+        layer(torch.zeros((4, in_f + 128), dtype=torch.float16, device="cuda"))
+    with pytest.raises(TypeError):
+        layer(torch.zeros((4, in_f), dtype=torch.float32, device="cuda"))
+    assert B.paro_fault_status() == 0

@@ -91,3 +91,20 @@ def test_pack_size_group_64(L):
     assert sb == 6144 // 16 * 64 * 8 * 4 and zb == 6144 // 16 * 64 * 8
     # 0.5 + 2/64 + 0.5/64 bytes per weight
     assert (qb + sb + zb) / (4096 * 6144) == pytest.approx(0.5 + 2 / 64 + 0.5 / 64)
+
+
+def test_prepared_layer_checks_its_arguments_once_on_the_host(L):
+    """ParoLinear refuses host tensors and a rotation prepared for another
+    group size or width before anything reaches the device."""
+    import torch
+    from rotated_w4_linear_b200 import binding
+    u8 = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        binding.ParoLinear(None, u8, u8, u8, 128, 16)
+
+    class FakeRot:                        # a handle-shaped stand-in; never passed to the library
+        group, in_features, handle = 64, 256, None
+    with pytest.raises(ValueError):
+        binding.ParoLinear(FakeRot(), u8, u8, u8, 256, 16, group=128)
+    with pytest.raises(ValueError):
+        binding.ParoLinear(FakeRot(), u8, u8, u8, 384, 16, group=64)

@@ -395,6 +395,9 @@ GemmArgs make_args(int64_t T, int64_t in, int64_t out, int group, const void* sc
     a.Gp = a.G + (a.G & 1);
     a.nkb = (int)(in / 64);
     a.nrb = (int)(out / 16);
+    // the kernel can split k over a cluster along z (16-token tiles, partial
+    // tiles reduced through distributed shared memory); the token tiles used
+    // here (64, 128, 256) need no split, so every launch runs one
     a.kb_per_split = a.nkb;
     a.nsplit = 1;
     a.sp = static_cast<const uint32_t*>(scp);

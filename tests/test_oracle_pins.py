@@ -309,3 +309,60 @@ def test_fp16_pipeline_golden():
     assert rdb.astype(np.float64).reshape(-1).tolist() == rows["rounded_bias"]
     # the exact layer does not round X': the ties above do not arise there
     assert np.allclose(O.linear(*layer).reshape(-1), rows["exact"], rtol=0, atol=1e-15)
+
+
+# ---- the other group sizes (CSDN article, section 5.2: 64 and 256) ---------
+@pytest.mark.parametrize("group", [64, 256])
+def test_group_sizes_keep_the_structure(group):
+    """At group 64 and 256: the rotation stays inside each group (a vector
+    nonzero in one group only stays so), preserves each group's norm when
+    alpha = 1, and (X T^-1)(T W) = X W; pairs reaching across a group are
+    refused."""
+    in_f = 512
+    pairs, theta, alpha = synth.rotation_params(in_f, 8, seed=group, pairs_per_group=group // 2, group=group)
+    x = synth.activations(6, in_f, seed=group).astype(np.float64)
+    ones = np.ones(in_f, np.float32)
+    xr = O.rotate_activations(x, pairs, theta, ones, group)
+    G = in_f // group
+    assert np.allclose(np.linalg.norm(x.reshape(6, G, group), axis=2), np.linalg.norm(xr.reshape(6, G, group), axis=2),
+                       rtol=1e-13)
+    one = np.zeros((1, in_f))
+    one[0, group:2 * group] = x[0, group:2 * group]
+    r1 = O.rotate_activations(one, pairs, theta, alpha, group)
+    assert np.all(r1[0, :group] == 0) and np.all(r1[0, 2 * group:] == 0) and np.any(r1[0, group:2 * group] != 0)
+    w = synth.weight(32, in_f, seed=group).astype(np.float64)
+    lhs = O.rotate_activations(x, pairs, theta, alpha, group) @ O.transform_weight(w, pairs, theta, alpha, group).T
+    assert np.linalg.norm(lhs - x @ w.T) / np.linalg.norm(x @ w.T) < 1e-12
+    bad = pairs.copy()
+    bad[0, 0, 0] = (0, group)                         # channel index outside its group
+    with pytest.raises(AssertionError):
+        O.rotate_activations(np.zeros((1, in_f)), bad, theta, alpha, group)
+
+
+@pytest.mark.parametrize("group", [64, 256])
+def test_group_sizes_pairwise_match_the_dense_matrix(group):
+    """Pairwise application against the independently built dense
+    block-diagonal T, at the real group sizes (two groups)."""
+    in_f = 2 * group
+    pairs, theta, alpha = synth.rotation_params(in_f, 4, seed=group + 1, pairs_per_group=group // 2, group=group)
+    T = O.dense_transform(pairs, theta, alpha, group=group)
+    assert np.all(T[:group, group:] == 0) and np.all(T[group:, :group] == 0)
+    x = np.random.default_rng(group).standard_normal((3, in_f))
+    assert np.allclose(O.rotate_activations(x, pairs, theta, alpha, group), x @ np.linalg.inv(T), atol=1e-11)
+
+
+@pytest.mark.parametrize("group", [64, 256])
+def test_rtn_invariants_other_group_sizes(group):
+    w = synth.weight(16, 512, seed=group).astype(np.float64)
+    q, s, z = O.rtn_quantize(w, group=group)
+    assert s.shape == (16, 512 // group) and z.shape == s.shape
+    sf = np.repeat(s.astype(np.float64), group, axis=1)
+    zf = np.repeat(z.astype(np.float64), group, axis=1)
+    exact = (q - zf) * sf
+    unclipped = (q > 0) & (q < 15)
+    assert np.all(np.abs(w - exact)[unclipped] <= sf[unclipped] / 2 * (1 + 1e-12))
+    # w_hat is the fp16 value nearest the exact product: within half the
+    # spacing above |w_hat| (the larger one where w_hat sits on a power of two)
+    wh = O.dequantize(q, s, z, group=group).astype(np.float64)
+    spacing = np.spacing(np.abs(wh).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(wh - exact) <= spacing / 2)

@@ -98,3 +98,20 @@ def test_traffic_figure_follows_the_kernel_source(monkeypatch):
     assert bench.gemv_traffic(4, "llama3-8b") is None
     monkeypatch.setattr(bench, "GEMV_TRAFFIC_SOURCE", "0" * 16)
     assert bench.gemv_traffic(16, "llama3-8b") is None
+
+
+def test_algorithmic_bytes_per_weight(monkeypatch):
+    """The bench's byte counts: 4-bit codes plus one fp16 scale and one
+    4-bit zero per group (0.5195 B per weight at group 128), the rotation's
+    parameters as the pages give them (per pair an fp32 cos/sin pair and
+    two channel bytes, 1/alpha per channel), and X read plus Y written."""
+    sys.path.insert(0, ROOT)
+    import bench
+    n_in, n_out = 4096, 4096
+    for g, per_weight in [(128, 0.5 + 2 / 128 + 0.5 / 128), (64, 0.5 + 2 / 64 + 0.5 / 64),
+                          (256, 0.5 + 2 / 256 + 0.5 / 256)]:
+        assert bench.weight_bytes(n_in, n_out, group=g) == n_in * n_out * per_weight
+    monkeypatch.setattr(bench, "GROUP", 128)
+    assert bench.rot_param_bytes(n_in, K=8, P=64) == 8 * 32 * 64 * 10 + 4 * 4096
+    assert bench.call_bytes(16, n_in, n_out) == (bench.weight_bytes(n_in, n_out) + 2 * 16 * (n_in + n_out)
+                                                 + bench.rot_param_bytes(n_in))
